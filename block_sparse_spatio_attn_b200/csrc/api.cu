@@ -1,0 +1,390 @@
+// api.cu -- the C entry points of svga.h: validation, sizes and launches.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "svga_internal.h"
+
+namespace svga {
+
+namespace {
+thread_local char g_last_error[512] = "";
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace
+
+void set_error(const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+static bool valid_tile(int t) { return t == 64 || t == 128 || t == 256; }
+
+// Shape checks shared by every call that takes a problem; per-head arrays are checked
+// only when need_heads is set.
+static svga_status validate_shape(const svga_problem *p, Geometry *g, bool need_heads)
+{
+    if (!p) {
+        set_error("problem is NULL");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (p->heads < 1 || p->heads > kMaxHeads) {
+        set_error("heads = %d outside 1..%d", p->heads, kMaxHeads);
+        return SVGA_ERR_SHAPE;
+    }
+    if (p->num_frames < 1 || p->grid_h < 1 || p->grid_w < 1 || p->num_frames > 65535) {
+        set_error("frames %d and grid %dx%d must be positive (frames <= 65535)", p->num_frames,
+                  p->grid_h, p->grid_w);
+        return SVGA_ERR_SHAPE;
+    }
+    const long long S = (long long)p->grid_h * p->grid_w;
+    const long long N = S * p->num_frames;
+    if (S > 65535 || N > kMaxTokens) {
+        set_error("tokens per frame %lld (max 65535) or tokens %lld (max %d) too large", S, N,
+                  kMaxTokens);
+        return SVGA_ERR_SHAPE;
+    }
+    if (p->head_dim != 64 && p->head_dim != 128) {
+        set_error("head_dim %d unsupported (64 or 128)", p->head_dim);
+        return SVGA_ERR_UNSUPPORTED;
+    }
+    if (p->anchor_frame0 != 0 && p->anchor_frame0 != 1) {
+        set_error("anchor_frame0 must be 0 or 1");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!valid_tile(p->tile_q) || !valid_tile(p->tile_k)) {
+        set_error("tile %dx%d unsupported (64, 128 or 256)", p->tile_q, p->tile_k);
+        return SVGA_ERR_UNSUPPORTED;
+    }
+    if (need_heads) {
+        if (!p->head_type || !p->band || !p->order) {
+            set_error("head_type, band and order must be host arrays of `heads` entries");
+            return SVGA_ERR_INVALID_ARG;
+        }
+        for (int h = 0; h < p->heads; ++h) {
+            if (p->head_type[h] != SVGA_HEAD_SPATIAL && p->head_type[h] != SVGA_HEAD_TEMPORAL) {
+                set_error("head %d: head_type %d invalid", h, p->head_type[h]);
+                return SVGA_ERR_INVALID_ARG;
+            }
+            if (p->band[h] < 0 || p->band[h] > 65535) {
+                set_error("head %d: band %d outside 0..65535", h, p->band[h]);
+                return SVGA_ERR_INVALID_ARG;
+            }
+            if (p->order[h] < SVGA_ORDER_FRAME_MAJOR || p->order[h] > SVGA_ORDER_TEMPORAL_MAJOR_STRICT) {
+                set_error("head %d: order %d invalid", h, p->order[h]);
+                return SVGA_ERR_INVALID_ARG;
+            }
+        }
+    }
+    g->heads = p->heads;
+    g->F = p->num_frames;
+    g->S = (int)S;
+    g->N = (int)N;
+    g->d = p->head_dim;
+    g->tile_q = p->tile_q;
+    g->tile_k = p->tile_k;
+    g->n_q = ceil_div(N, p->tile_q);
+    g->n_k = ceil_div(N, p->tile_k);
+    g->kn = p->tile_k < 128 ? p->tile_k : 128;
+    g->n_qblk = ceil_div(N, kBlockM);
+    g->n_pairs = ceil_div(g->n_qblk, 2);
+    g->n_kc = ceil_div(N, g->kn);
+    g->n_items = g->heads * g->n_pairs;
+    return SVGA_OK;
+}
+
+svga_status validate_problem(const svga_problem *p, Geometry *g) { return validate_shape(p, g, true); }
+
+size_t plan_header_bytes(const Geometry &g)
+{
+    return align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)g.heads + g.n_items), 256);
+}
+
+int64_t plan_entry_cap(const Geometry &g) { return (int64_t)g.n_items * g.n_kc; }
+
+static svga_status check_tensor(const void *p, const char *name)
+{
+    if (!p) {
+        set_error("%s is NULL", name);
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!aligned(p, 16)) {
+        set_error("%s is not 16-byte aligned", name);
+        return SVGA_ERR_ALIGNMENT;
+    }
+    return SVGA_OK;
+}
+
+static svga_status check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error("%s: %s", what, cudaGetErrorString(e));
+        return SVGA_ERR_CUDA;
+    }
+    return SVGA_OK;
+}
+
+}  // namespace svga
+
+using namespace svga;
+
+extern "C" {
+
+svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes, size_t *ptr_bytes,
+                                int64_t *full_cap, int64_t *bnd_cap, size_t *plan_bytes,
+                                size_t *workspace_bytes)
+{
+    Geometry g;
+    svga_status rc = validate_problem(problem, &g);
+    if (rc != SVGA_OK) return rc;
+    const int64_t tiles = (int64_t)g.heads * g.n_q * g.n_k;
+    if (cls_bytes) *cls_bytes = (size_t)tiles;
+    if (ptr_bytes) *ptr_bytes = sizeof(int32_t) * ((size_t)g.heads * g.n_q + 1);
+    if (full_cap) *full_cap = tiles;
+    if (bnd_cap) *bnd_cap = tiles;
+    if (plan_bytes) *plan_bytes = plan_header_bytes(g) + sizeof(uint32_t) * (size_t)plan_entry_cap(g);
+    if (workspace_bytes) *workspace_bytes = block_map_workspace_bytes(g);
+    return SVGA_OK;
+}
+
+svga_status svga_build_block_map(const svga_problem *problem, svga_block_map *map, void *workspace,
+                                 size_t workspace_bytes, svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_problem(problem, &g);
+    if (rc != SVGA_OK) return rc;
+    if (!map || !map->cls || !map->full_ptr || !map->full_idx || !map->bnd_ptr || !map->bnd_idx ||
+        !map->plan || !workspace) {
+        set_error("block map buffers and workspace must be non-NULL device pointers");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!aligned(map->plan, 256) || !aligned(workspace, 256) || !aligned(map->full_ptr, 4) ||
+        !aligned(map->bnd_ptr, 4) || !aligned(map->full_idx, 4) || !aligned(map->bnd_idx, 4)) {
+        set_error("plan and workspace must be 256-byte aligned, CSR arrays 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (workspace_bytes < block_map_workspace_bytes(g) || map->plan_bytes < plan_header_bytes(g) ||
+        map->full_cap < 0 || map->bnd_cap < 0) {
+        set_error("workspace (%zu < %zu) or plan (%zu) smaller than svga_block_map_size",
+                  workspace_bytes, block_map_workspace_bytes(g), map->plan_bytes);
+        return SVGA_ERR_WORKSPACE;
+    }
+    return launch_build_block_map(problem, g, map, workspace, workspace_bytes, stream);
+}
+
+static svga_status permute_common(const void *src, void *dst, const svga_problem *problem,
+                                  svga_stream_t stream, int inverse)
+{
+    Geometry g;
+    svga_status rc = validate_problem(problem, &g);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_tensor(src, "src")) != SVGA_OK || (rc = check_tensor(dst, "dst")) != SVGA_OK)
+        return rc;
+    const size_t bytes = (size_t)g.heads * g.N * g.d * 2;
+    const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
+    if (s < d + bytes && d < s + bytes) {
+        set_error("src and dst overlap");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    return launch_permute(src, dst, problem, g, inverse, stream);
+}
+
+svga_status svga_permute_tokens(const void *src, void *dst, const svga_problem *problem,
+                                svga_stream_t stream)
+{
+    return permute_common(src, dst, problem, stream, 0);
+}
+
+svga_status svga_unpermute_tokens(const void *src, void *dst, const svga_problem *problem,
+                                  svga_stream_t stream)
+{
+    return permute_common(src, dst, problem, stream, 1);
+}
+
+svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                                      float *lse, const svga_problem *problem,
+                                      const svga_block_map *map, float scale, int flags,
+                                      svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_problem(problem, &g);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
+        (rc = check_tensor(v, "v")) != SVGA_OK || (rc = check_tensor(o, "o")) != SVGA_OK)
+        return rc;
+    if (lse && !aligned(lse, 4)) {
+        set_error("lse is not 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (!map || !map->plan || map->plan_bytes < plan_header_bytes(g)) {
+        set_error("block map plan missing or smaller than svga_block_map_size");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (flags & ~SVGA_FLAG_NAIVE_B1) {
+        set_error("unknown flags 0x%x", flags);
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!(scale > 0.f) || !(scale < 1e30f)) {
+        set_error("scale must be a positive finite number");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (map->status && cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess)
+        return check_launch("cudaMemsetAsync(status)");
+    AttnLaunch a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.lse = lse;
+    a.heads = g.heads;
+    a.nq_rows = g.N;
+    a.nk_rows = g.N;
+    a.d = g.d;
+    a.F = g.F;
+    a.S = g.S;
+    a.anchor = problem->anchor_frame0;
+    a.scale = scale;
+    a.mode = 0;
+    a.naive = (flags & SVGA_FLAG_NAIVE_B1) ? 1 : 0;
+    a.kn = g.kn;
+    a.plan = map->plan;
+    a.n_items = g.n_items;
+    a.status = map->status;
+    return launch_attention(a, stream);
+}
+
+svga_status svga_dense_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                                     float *lse, int heads, int tokens, int head_dim, float scale,
+                                     int32_t *status, svga_stream_t stream)
+{
+    if (heads < 1 || heads > kMaxHeads || tokens < 1 || tokens > kMaxTokens) {
+        set_error("heads %d / tokens %d outside 1..%d / 1..%d", heads, tokens, kMaxHeads,
+                  kMaxTokens);
+        return SVGA_ERR_SHAPE;
+    }
+    if (head_dim != 64 && head_dim != 128) {
+        set_error("head_dim %d unsupported (64 or 128)", head_dim);
+        return SVGA_ERR_UNSUPPORTED;
+    }
+    svga_status rc;
+    if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
+        (rc = check_tensor(v, "v")) != SVGA_OK || (rc = check_tensor(o, "o")) != SVGA_OK)
+        return rc;
+    if (lse && !aligned(lse, 4)) {
+        set_error("lse is not 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (!(scale > 0.f) || !(scale < 1e30f)) {
+        set_error("scale must be a positive finite number");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (status && cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess)
+        return check_launch("cudaMemsetAsync(status)");
+    AttnLaunch a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.lse = lse;
+    a.heads = heads;
+    a.nq_rows = tokens;
+    a.nk_rows = tokens;
+    a.d = head_dim;
+    a.F = 1;
+    a.S = tokens;
+    a.scale = scale;
+    a.mode = 1;
+    a.kn = 128;
+    const int n_qblk = (tokens + kBlockM - 1) / kBlockM;
+    a.n_items = heads * ((n_qblk + 1) / 2);
+    a.status = status;
+    return launch_attention(a, stream);
+}
+
+svga_status svga_classify_size(const svga_problem *problem, int n_rows, size_t *workspace_bytes)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, false);
+    if (rc != SVGA_OK) return rc;
+    if (n_rows < 1 || n_rows > g.N) {
+        set_error("n_rows %d outside 1..%d", n_rows, g.N);
+        return SVGA_ERR_SHAPE;
+    }
+    if (workspace_bytes) *workspace_bytes = classify_workspace_bytes(problem, n_rows);
+    return SVGA_OK;
+}
+
+svga_status svga_classify_heads(const void *q, const void *k, const void *v,
+                                const svga_problem *problem, const int32_t *w_spatial,
+                                const int32_t *w_temporal, const int32_t *rows, int n_rows,
+                                float scale, int32_t *head_type_out, float *mse_out,
+                                void *workspace, size_t workspace_bytes, svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, false);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
+        (rc = check_tensor(v, "v")) != SVGA_OK)
+        return rc;
+    if (n_rows < 1 || n_rows > g.N) {
+        set_error("n_rows %d outside 1..%d", n_rows, g.N);
+        return SVGA_ERR_SHAPE;
+    }
+    if (!w_spatial || !w_temporal || !head_type_out) {
+        set_error("w_spatial, w_temporal and head_type_out must be host arrays");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    for (int h = 0; h < g.heads; ++h)
+        if (w_spatial[h] < 0 || w_spatial[h] > 65535 || w_temporal[h] < 0 || w_temporal[h] > 65535) {
+            set_error("head %d: candidate bands must be in 0..65535", h);
+            return SVGA_ERR_INVALID_ARG;
+        }
+    if (rows && !aligned(rows, 4)) {
+        set_error("rows is not 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (!(scale > 0.f) || !(scale < 1e30f)) {
+        set_error("scale must be a positive finite number");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!workspace || !aligned(workspace, 256) ||
+        workspace_bytes < classify_workspace_bytes(problem, n_rows)) {
+        set_error("workspace missing, not 256-byte aligned or smaller than svga_classify_size");
+        return SVGA_ERR_WORKSPACE;
+    }
+    return run_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
+                        head_type_out, mse_out, workspace, workspace_bytes, stream);
+}
+
+const char *svga_last_error(void) { return g_last_error; }
+
+const char *svga_status_string(svga_status s)
+{
+    switch (s) {
+    case SVGA_OK: return "SVGA_OK";
+    case SVGA_ERR_INVALID_ARG: return "SVGA_ERR_INVALID_ARG";
+    case SVGA_ERR_SHAPE: return "SVGA_ERR_SHAPE";
+    case SVGA_ERR_ALIGNMENT: return "SVGA_ERR_ALIGNMENT";
+    case SVGA_ERR_UNSUPPORTED: return "SVGA_ERR_UNSUPPORTED";
+    case SVGA_ERR_WORKSPACE: return "SVGA_ERR_WORKSPACE";
+    case SVGA_ERR_CUDA: return "SVGA_ERR_CUDA";
+    case SVGA_ERR_TIMEOUT: return "SVGA_ERR_TIMEOUT";
+    }
+    return "unknown svga_status";
+}
+
+int svga_version(void) { return SVGA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,607 @@
+// attention.cu -- block-sparse flash-attention forward for B200 (sm_100a).
+//
+// Computes, per head and query row, the masked softmax(scale * q k^T) v over the keys
+// the head's mask keeps, walking only the key tiles that hold kept pairs.  Full tiles
+// run with no mask arithmetic; boundary tiles are masked element by element from the
+// tokens' (frame, in-frame index) coordinates.  This is the full/boundary tile
+// specialisation of "Accelerating Spatio-Temporal Attention for Video Diffusion on
+// TPUs" (aihirek.info, section "A TPU-kernel kialakitasa dontonek bizonyult";
+// ainews.tenesys.com, "Co sie zmienilo?" items 1-2), written for Blackwell:
+//
+//   * one CTA per work item = two consecutive 128-row query blocks (Q0, Q1) that share
+//     one stream of key chunks (the merged lists of the two blocks);
+//   * warp 0 streams K and V chunks with TMA (128-byte swizzle) through a ring of
+//     shared-memory stages; warp 1 issues tcgen05.mma from one thread:
+//       S_i = Q_i K^T  (A, B from shared memory, D in TMEM, fp32)
+//       O_i += P_i V   (A = P from TMEM as bf16, B = V from shared memory)
+//     in the order S0(n+1) after PV0(n) and S1(n+1) after PV1(n), so the two softmax
+//     warpgroups work on different tiles while the tensor core runs the other's MMAs;
+//   * warps 4-7 and 8-11 hold one query row per thread (TMEM lane = row): they read S,
+//     apply the mask on boundary tiles, run the online softmax in the exp2 domain,
+//     write P back into TMEM over S, and rescale O in TMEM only when the running
+//     maximum grows by more than 2^8 (P stays <= 256 otherwise);
+//   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated).
+//
+// Every mbarrier wait gives up after about a second: the CTA raises a shared abort
+// flag, drains its MMAs and copies, frees TMEM, writes SVGA_ERR_TIMEOUT to the
+// caller's status word and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "svga_device.cuh"
+#include "svga_internal.h"
+
+namespace svga {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct KParams {
+    int heads, nq_rows, nk_rows, F, S, anchor;
+    float scale_log2;
+    int mode, naive, n_pairs, n_qblk, n_kc;
+    const int4 *items;
+    const uint32_t *entries;
+    const int4 *head_info;
+    const int32_t *qrow_tokens;
+    void *o;
+    float *lse;
+    int32_t *status;
+};
+
+template <int D, int KN>
+struct Cfg {
+    static constexpr int kQBytes = kBlockM * D * 2;             // one 128-row Q tile
+    static constexpr int kQChunk = kBlockM * 128;               // 64 columns x 128 rows
+    static constexpr int kKVBytes = KN * D * 2;                  // one K or V chunk
+    static constexpr int kKVChunk = KN * 128;                    // 64 columns x KN rows
+    static constexpr int kStages = (kKVBytes >= 32768) ? 4 : 8;
+    static constexpr int kSmemData = 2 * kQBytes + kStages * kKVBytes;
+    static constexpr int kSmemBar = 1024;
+    static constexpr int kSmemAlloc = kSmemData + kSmemBar + 1024;  // + alignment slack
+    static constexpr int kSmemLaunch = kSmemAlloc < 120 * 1024 ? 120 * 1024 : kSmemAlloc;
+    static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+};
+
+struct Barriers {
+    uint64_t q_full;
+    uint64_t kv_full[8];
+    uint64_t kv_empty[8];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct Item {
+    int h, b0, E;
+    const uint32_t *ent;
+    bool valid1, ragged;
+    int mode, naive, n_kc;
+
+    __device__ __forceinline__ uint32_t entry(int n) const
+    {
+        if (mode == 0) {
+            uint32_t e = __ldg(ent + n);
+            if (naive) e &= ~(kEntF0 | kEntF1);
+            return e;
+        }
+        const bool full = (mode == 1) && !(ragged && n == n_kc - 1);
+        uint32_t e = (uint32_t)n | kEntV0 | (full ? kEntF0 : 0u);
+        if (valid1) e |= kEntV1 | (full ? kEntF1 : 0u);
+        return e;
+    }
+};
+
+__device__ __forceinline__ Item make_item(const KParams &p)
+{
+    Item it;
+    it.mode = p.mode;
+    it.naive = p.naive;
+    it.n_kc = p.n_kc;
+    if (p.mode == 0) {
+        const int4 x = __ldg(p.items + blockIdx.x);
+        it.h = x.x;
+        it.b0 = x.y;
+        it.ent = p.entries + x.z;
+        it.E = x.w;
+    } else {
+        it.h = blockIdx.x / p.n_pairs;
+        it.b0 = 2 * (blockIdx.x - it.h * p.n_pairs);
+        it.ent = nullptr;
+        it.E = p.n_kc;
+    }
+    it.valid1 = it.b0 + 1 < p.n_qblk;
+    return it;
+}
+
+// Advance (f, s) to the next position of `order`.
+__device__ __forceinline__ void step_coord(int order, int F, int S, int &f, int &s)
+{
+    if (order == ORDER_FM) {
+        if (++s == S) {
+            s = 0;
+            ++f;
+        }
+    } else if (order == ORDER_TM_STRICT) {
+        if (++f == F) {
+            f = 0;
+            ++s;
+        }
+    } else {
+        if (f == 0) {
+            if (++s == S) {
+                s = 0;
+                f = 1;
+            }
+        } else if (++f == F) {
+            f = 1;
+            ++s;
+        }
+    }
+}
+
+template <int D, int KN, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const KParams p)
+{
+    using C = Cfg<D, KN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint8_t *sQ = smem;                                  // 2 x kQBytes
+    uint8_t *sKV = smem + 2 * C::kQBytes;                // kStages x kKVBytes
+    Barriers *bar = reinterpret_cast<Barriers *>(smem + C::kSmemData);
+    volatile int *abort_flag = &bar->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Item it = make_item(p);
+    it.ragged = (p.nk_rows % KN) != 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar->q_full), 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&bar->kv_full[s]), 1);
+            mbar_init(smem_u32(&bar->kv_empty[s]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bar->s_full[i]), 1);
+            mbar_init(smem_u32(&bar->p_full[i]), 128);
+            mbar_init(smem_u32(&bar->o_done[i]), 1);
+        }
+        mbar_init(smem_u32(&bar->drain), 1);
+        bar->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bar->tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            const uint32_t qf = smem_u32(&bar->q_full);
+            mbar_arrive_expect_tx(qf, (it.valid1 ? 2 : 1) * C::kQBytes);
+            for (int i = 0; i < (it.valid1 ? 2 : 1); ++i)
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(smem_u32(sQ + i * C::kQBytes + c * C::kQChunk), &tmQ, qf, 64 * c,
+                                (it.b0 + i) * kBlockM, it.h);
+            int issued = 0;
+            bool ok = true;
+            for (int n = 0; n < it.E && ok; ++n) {
+                const int kc = (int)(it.entry(n) & kEntChunkMask);
+                for (int t = 0; t < 2; ++t) {
+                    const int idx = 2 * n + t, s = idx % C::kStages, round = idx / C::kStages;
+                    if (round > 0 &&
+                        !mbar_wait(smem_u32(&bar->kv_empty[s]), (round - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&bar->kv_full[s]);
+                    mbar_arrive_expect_tx(fb, C::kKVBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(smem_u32(sKV + s * C::kKVBytes + c * C::kKVChunk),
+                                    t ? &tmV : &tmK, fb, 64 * c, kc * KN, it.h);
+                    issued = idx + 1;
+                }
+            }
+            if (!ok) {
+                // Abort: let the copies in flight land before the CTA exits.
+                mbar_wait_bounded(qf, 0);
+                for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
+                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
+                                      (idx / C::kStages) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        constexpr uint32_t idS = idesc_bf16_f32(kBlockM, KN, 0);
+        constexpr uint32_t idO = idesc_bf16_f32(kBlockM, D, 1);
+        const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->q_full), 0, abort_flag));
+        tc_fence_after();
+        const int total = 2 * it.E;
+        auto wait_full = [&](int idx) {
+            const int s = idx % C::kStages;
+            bool r = __all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&bar->kv_full[s]), (idx / C::kStages) & 1,
+                                          abort_flag));
+            tc_fence_after();
+            return r;
+        };
+        auto issue_s = [&](int i, int idx) {
+            const uint32_t a0 = sQa + i * C::kQBytes, b0 = sKVa + (idx % C::kStages) * C::kKVBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off_a = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
+                const uint32_t off_b = (kk >> 2) * C::kKVChunk + (kk & 3) * 32;
+                mma_ss(tmem + i * 128, smem_desc_sw128(a0 + off_a, 16, 1024),
+                       smem_desc_sw128(b0 + off_b, 16, 1024), idS, kk > 0);
+            }
+            mma_commit(smem_u32(&bar->s_full[i]));
+        };
+        auto issue_pv = [&](int i, int idx, bool first) {
+            const uint32_t b0 = sKVa + (idx % C::kStages) * C::kKVBytes;
+#pragma unroll
+            for (int kk = 0; kk < KN / 16; ++kk)
+                mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
+                       smem_desc_sw128(b0 + kk * 2048, C::kKVChunk, 1024), idO,
+                       (!first || kk > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&bar->o_done[i]));
+        };
+        auto release = [&](int idx) {
+            if (idx + C::kStages < total) mma_commit(smem_u32(&bar->kv_empty[idx % C::kStages]));
+        };
+        int pv[2] = {0, 0};
+        if (ok && it.E > 0) {
+            const uint32_t e0 = it.entry(0);
+            ok = wait_full(0);
+            if (ok && lane == 0) {
+                if (e0 & kEntV0) issue_s(0, 0);
+                if (e0 & kEntV1) issue_s(1, 0);
+                release(0);
+            }
+            __syncwarp();
+        }
+        for (int n = 0; ok && n < it.E; ++n) {
+            const uint32_t e = it.entry(n);
+            const bool has_next = n + 1 < it.E;
+            const uint32_t en = has_next ? it.entry(n + 1) : 0u;
+            if (!(ok = wait_full(2 * n + 1))) break;
+            if (e & kEntV0) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&bar->p_full[0]), pv[0] & 1, abort_flag));
+                tc_fence_after();
+                if (!ok) break;
+                if (lane == 0) issue_pv(0, 2 * n + 1, pv[0] == 0);
+                ++pv[0];
+            }
+            if (has_next) {
+                if (!(ok = wait_full(2 * n + 2))) break;
+                if (lane == 0 && (en & kEntV0)) issue_s(0, 2 * n + 2);
+            }
+            if (e & kEntV1) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&bar->p_full[1]), pv[1] & 1, abort_flag));
+                tc_fence_after();
+                if (!ok) break;
+                if (lane == 0) issue_pv(1, 2 * n + 1, pv[1] == 0);
+                ++pv[1];
+            }
+            if (lane == 0) {
+                if (has_next) {
+                    if (en & kEntV1) issue_s(1, 2 * n + 2);
+                    release(2 * n + 2);
+                }
+                release(2 * n + 1);
+            }
+            __syncwarp();
+        }
+        if (!ok) {
+            // Abort: wait for every MMA issued so far before TMEM is freed.
+            if (lane == 0) mma_commit(smem_u32(&bar->drain));
+            __syncwarp();
+            mbar_wait_bounded(smem_u32(&bar->drain), 0);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------ softmax warpgroups
+        const int wg = (warp - 4) >> 2, quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const uint32_t tS = tmem + lane_base + wg * 128;
+        const uint32_t tO = tmem + lane_base + 256 + wg * 128;
+        const int blk = it.b0 + wg;
+        const int qpos = blk * kBlockM + row;
+        const bool row_valid = qpos < p.nq_rows;
+        int type = MASK_DENSE, band = 0, korder = ORDER_FM;
+        if (p.mode != 1) {
+            const int4 hi = __ldg(p.head_info + it.h);
+            type = hi.x;
+            band = hi.y;
+            korder = hi.z;
+        }
+        int fq = 0, sq = 0;
+        if (row_valid && type != MASK_DENSE) {
+            if (p.qrow_tokens) {
+                const int t = __ldg(p.qrow_tokens + qpos);
+                fq = t / p.S;
+                sq = t - fq * p.S;
+            } else {
+                pos_to_coord(korder, qpos, p.F, p.S, fq, sq);
+            }
+        }
+        const uint32_t vbit = wg ? kEntV1 : kEntV0, fbit = wg ? kEntF1 : kEntF0;
+        float m_used = -INFINITY, l = 0.f;
+        int visit = 0;
+        bool ok = true;
+        for (int n = 0; n < it.E; ++n) {
+            const uint32_t e = it.entry(n);
+            if (!(e & vbit)) continue;
+            const bool full = (e & fbit) != 0;
+            const int kc = (int)(e & kEntChunkMask);
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&bar->s_full[wg]), visit & 1, abort_flag));
+            tc_fence_after();
+            if (!ok) break;
+            uint32_t r[KN];
+#pragma unroll
+            for (int j = 0; j < KN / 32; ++j)
+                tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[j * 32]));
+            tmem_wait_ld();
+            if (!full) {
+                const int k0 = kc * KN;
+                int fk = 0, sk = 0;
+                pos_to_coord(korder, min(k0, p.nk_rows - 1), p.F, p.S, fk, sk);
+#pragma unroll
+                for (int c = 0; c < KN; ++c) {
+                    bool keep = (k0 + c) < p.nk_rows;
+                    if (type != MASK_DENSE)
+                        keep = keep && keep_pair(type, band, p.anchor, fq, sq, fk, sk);
+                    if (!keep) r[c] = __float_as_uint(-INFINITY);
+                    step_coord(korder, p.F, p.S, fk, sk);
+                }
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < KN; c += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(r[c]));
+                mx1 = fmaxf(mx1, __uint_as_float(r[c + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(r[c + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(r[c + 3]));
+            }
+            const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+            bool need = false;
+            float m_new;
+            if (m_used == -INFINITY) {
+                m_used = m_new = mt;  // O holds only zero rows so far: nothing to rescale
+            } else if (mt > m_used + kRescaleThreshold) {
+                need = true;
+                m_new = mt;
+            } else {
+                m_new = m_used;
+            }
+            if (__any_sync(0xffffffffu, need)) {
+                // O += P V of the previous visit must be complete before O is touched.
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->o_done[wg]),
+                                                       (visit - 1) & 1, abort_flag));
+                tc_fence_after();
+                if (!ok) break;
+                const float fac = need ? fast_exp2(m_used - m_new) : 1.f;
+                l *= fac;
+                m_used = m_new;
+#pragma unroll 1
+                for (int j = 0; j < D / 32; ++j) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + j * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
+                    tmem_st32(tO + j * 32, o);
+                }
+                tmem_wait_st();
+            }
+            const float ms = (m_used == -INFINITY) ? 0.f : m_used;
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < KN / 64; ++j) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float a = fast_exp2(fmaf(__uint_as_float(r[j * 64 + 2 * c]), p.scale_log2, -ms));
+                    const float b = fast_exp2(fmaf(__uint_as_float(r[j * 64 + 2 * c + 1]), p.scale_log2, -ms));
+                    sum0 += a;
+                    sum1 += b;
+                    pk[c] = pack_bf16x2(a, b);
+                }
+                tmem_st32(tS + j * 32, pk);
+            }
+            tmem_wait_st();
+            l += sum0 + sum1;
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bar->p_full[wg]));
+            ++visit;
+        }
+        // ----------------------------------------------------------------- epilogue
+        if (ok && visit > 0) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&bar->o_done[wg]), (visit - 1) & 1, abort_flag));
+            tc_fence_after();
+        }
+        if (ok && (blk < p.n_qblk)) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t orow = ((size_t)it.h * p.nq_rows + (row_valid ? qpos : 0)) * D;
+#pragma unroll 1
+            for (int j = 0; j < D / 32; ++j) {
+                uint32_t o[32];
+                if (visit > 0) {
+                    tmem_ld32(tO + j * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
+                if (row_valid) {
+                    if (OUT_F32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + j * 32);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv,
+                                                 __uint_as_float(o[4 * c + 1]) * inv,
+                                                 __uint_as_float(o[4 * c + 2]) * inv,
+                                                 __uint_as_float(o[4 * c + 3]) * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow + j * 32);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            dst[c] = make_uint4(
+                                pack_bf16x2(__uint_as_float(o[8 * c]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+                    }
+                }
+            }
+            if (row_valid && p.lse)
+                p.lse[(size_t)it.h * p.nq_rows + qpos] =
+                    l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && bar->abort && p.status) atomicExch(p.status, (int32_t)SVGA_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// [heads, rows, d] bf16, box = 64 columns x box_rows rows x 1 head, 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *base, int heads, int rows, int d, int box_rows)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int KN, bool OUT_F32>
+svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
+{
+    using C = Cfg<D, KN>;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, a.q, a.heads, a.nq_rows, D, kBlockM) ||
+        !make_tmap(&tk, a.k, a.heads, a.nk_rows, D, KN) ||
+        !make_tmap(&tv, a.v, a.heads, a.nk_rows, D, KN)) {
+        set_error("cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+        return SVGA_ERR_CUDA;
+    }
+    auto kfn = attn_fwd_kernel<D, KN, OUT_F32>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) !=
+        cudaSuccess) {
+        set_error("cudaFuncSetAttribute(max dynamic shared memory) failed");
+        return SVGA_ERR_CUDA;
+    }
+    if (a.n_items > 0) kfn<<<a.n_items, kThreads, C::kSmemLaunch, st>>>(tq, tk, tv, kp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error("attention launch failed: %s", cudaGetErrorString(e));
+        return SVGA_ERR_CUDA;
+    }
+    return SVGA_OK;
+}
+
+}  // namespace
+
+svga_status launch_attention(const AttnLaunch &a, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    KParams kp{};
+    kp.heads = a.heads;
+    kp.nq_rows = a.nq_rows;
+    kp.nk_rows = a.nk_rows;
+    kp.F = a.F;
+    kp.S = a.S;
+    kp.anchor = a.anchor;
+    kp.scale_log2 = a.scale * kLog2e;
+    kp.mode = a.mode;
+    kp.naive = a.naive;
+    kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
+    kp.n_pairs = (kp.n_qblk + 1) / 2;
+    kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;
+    if (a.mode == 0) {
+        const char *plan = static_cast<const char *>(a.plan);
+        kp.head_info = reinterpret_cast<const int4 *>(plan + sizeof(PlanHeader));
+        kp.items = kp.head_info + a.heads;
+    } else {
+        kp.head_info = reinterpret_cast<const int4 *>(a.head_info);
+        kp.items = nullptr;
+        kp.entries = nullptr;
+    }
+    kp.qrow_tokens = a.qrow_tokens;
+    kp.o = a.o;
+    kp.lse = a.lse;
+    kp.status = a.status;
+    if (a.mode == 0) {
+        // entries start after header + head_info + items, 256-byte aligned
+        size_t hdr = sizeof(PlanHeader) + sizeof(int4) * ((size_t)a.heads + a.n_items);
+        hdr = align_up(hdr, 256);
+        kp.entries = reinterpret_cast<const uint32_t *>(static_cast<const char *>(a.plan) + hdr);
+    }
+    const int d = a.d, kn = a.kn;
+    if (d == 128 && kn == 128)
+        return a.out_f32 ? launch_t<128, 128, true>(a, kp, st) : launch_t<128, 128, false>(a, kp, st);
+    if (d == 128 && kn == 64)
+        return a.out_f32 ? launch_t<128, 64, true>(a, kp, st) : launch_t<128, 64, false>(a, kp, st);
+    if (d == 64 && kn == 128)
+        return a.out_f32 ? launch_t<64, 128, true>(a, kp, st) : launch_t<64, 128, false>(a, kp, st);
+    if (d == 64 && kn == 64)
+        return a.out_f32 ? launch_t<64, 64, true>(a, kp, st) : launch_t<64, 64, false>(a, kp, st);
+    set_error("unsupported head_dim %d / key chunk %d", d, kn);
+    return SVGA_ERR_UNSUPPORTED;
+}
+
+}  // namespace svga

@@ -1,0 +1,75 @@
+// permute.cu -- token permutation between frame-major and a head's token order.
+//
+// The pages move the tokens of temporal heads from frame-major to temporal-major
+// order so that a temporal head's band lines up with the tiles ("Accelerating
+// Spatio-Temporal Attention for Video Diffusion on TPUs", ainews.tenesys.com,
+// "Co sie zmienilo?" item 5).  Both directions are gathers: every thread writes one
+// 16-byte piece of a destination row (coalesced) and reads the matching piece of the
+// source row the order maps it to (a whole 128- or 256-byte row per warp quarter or
+// half, so reads stay full cache lines).  Pure data movement: bound by HBM bandwidth.
+#include <cuda_runtime.h>
+
+#include "svga_device.cuh"
+#include "svga_internal.h"
+
+namespace svga {
+namespace {
+
+struct OrderParams {
+    uint8_t order[kMaxHeads];
+};
+
+template <int VPR>  // 16-byte vectors per row (head_dim / 8)
+__global__ void __launch_bounds__(256) permute_kernel(const uint4 *__restrict__ src,
+                                                      uint4 *__restrict__ dst, int N, int F, int S,
+                                                      int inverse, OrderParams op)
+{
+    const int h = blockIdx.y;
+    const int order = op.order[h];
+    const size_t head_off = (size_t)h * N * VPR;
+    const int total = N * VPR;
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+        const int drow = idx / VPR, v = idx - drow * VPR;
+        int srow;
+        if (order == ORDER_FM) {
+            srow = drow;
+        } else if (!inverse) {
+            int f, s;
+            pos_to_coord(order, drow, F, S, f, s);  // dst position -> its token
+            srow = f * S + s;                       // token's frame-major row
+        } else {
+            const int f = drow / S, s = drow - f * S;  // dst is frame-major token
+            srow = coord_to_pos(order, f, s, F, S);    // where the order put it
+        }
+        dst[head_off + (size_t)drow * VPR + v] = __ldg(src + head_off + (size_t)srow * VPR + v);
+    }
+}
+
+}  // namespace
+
+svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
+                           int inverse, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    OrderParams op;
+    for (int h = 0; h < g.heads; ++h) op.order[h] = (uint8_t)p->order[h];
+    const int vpr = g.d / 8;
+    const int total = g.N * vpr;
+    int blocks = (total + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    dim3 grid(blocks, g.heads);
+    if (vpr == 16)
+        permute_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
+                                                 static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op);
+    else
+        permute_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
+                                                static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error("permute launch failed: %s", cudaGetErrorString(e));
+        return SVGA_ERR_CUDA;
+    }
+    return SVGA_OK;
+}
+
+}  // namespace svga

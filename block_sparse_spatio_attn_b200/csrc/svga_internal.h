@@ -1,0 +1,89 @@
+// svga_internal.h -- definitions shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/svga.h"
+
+namespace svga {
+
+// token orders (values of svga.h's SVGA_ORDER_*)
+enum { ORDER_FM = 0, ORDER_TM = 1, ORDER_TM_STRICT = 2 };
+// mask kinds used inside kernels (SVGA_HEAD_* plus dense)
+enum { MASK_SPATIAL = 0, MASK_TEMPORAL = 1, MASK_DENSE = 2 };
+
+constexpr int kMaxHeads = 4096;
+constexpr int kMaxTokens = 1 << 24;
+constexpr int kBlockM = 128;  // query rows per tcgen05 tile (one TMEM lane per row)
+
+// Execution plan of the attention kernel, stored in svga_block_map::plan.
+//   PlanHeader, then int4 head_info[heads] = {mask type, band, order, 0},
+//   then int4 items[n_items] = {head, first 128-row block, entry offset, entry count}
+//   in longest-first order, then uint32 entries[].
+// A work item is a pair of consecutive 128-row query blocks; an entry is one key
+// chunk of kn keys visited by at least one of the two blocks:
+//   bits 0-23 key chunk index, bit 24 block 0 visits, bit 25 block 0 full,
+//   bit 26 block 1 visits, bit 27 block 1 full.
+struct PlanHeader {
+    int32_t magic;
+    int32_t heads, tokens, frames, tokens_per_frame, anchor;
+    int32_t tile_q, tile_k, kn, n_qblk, n_kc, n_items;
+    int64_t entry_cap;
+    int32_t reserved[2];
+};
+static_assert(sizeof(PlanHeader) == 64, "plan header is 64 bytes");
+constexpr int32_t kPlanMagic = 0x53564741;  // "SVGA"
+
+constexpr uint32_t kEntChunkMask = 0x00FFFFFFu;
+constexpr uint32_t kEntV0 = 1u << 24, kEntF0 = 1u << 25, kEntV1 = 1u << 26, kEntF1 = 1u << 27;
+
+struct Geometry {
+    int heads, F, S, N, d;
+    int tile_q, tile_k, n_q, n_k;
+    int kn, n_qblk, n_pairs, n_kc, n_items;
+};
+
+// ----------------------------------------------------------- host-side helpers
+void set_error(const char *fmt, ...);
+svga_status validate_problem(const svga_problem *p, Geometry *g);
+size_t plan_header_bytes(const Geometry &g);  // header + head_info + items, 256-aligned
+int64_t plan_entry_cap(const Geometry &g);
+size_t align_up(size_t x, size_t a);
+
+// block_map.cu
+svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svga_block_map *map,
+                                   void *ws, size_t ws_bytes, void *stream);
+size_t block_map_workspace_bytes(const Geometry &g);
+
+// permute.cu
+svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
+                           int inverse, void *stream);
+
+// attention.cu
+struct AttnLaunch {
+    const void *q, *k, *v;
+    void *o;
+    float *lse;
+    int heads, nq_rows, nk_rows, d;
+    int F, S, anchor;
+    float scale;
+    int mode;                  // 0 plan, 1 dense (implicit), 2 masked everywhere (implicit)
+    int naive;                 // plan mode: visit full tiles through the masked path
+    int kn;                    // keys per chunk: 64 or 128
+    const void *plan;          // device plan (mode 0)
+    const int32_t *head_info;  // device int4 per head (modes 0 and 2)
+    const int32_t *qrow_tokens;  // device [nq_rows] frame-major token of each query row (shared by all heads) or null
+    int out_f32;               // o is float32 instead of bf16
+    int n_items;
+    int32_t *status;
+};
+svga_status launch_attention(const AttnLaunch &a, void *stream);
+
+// classify.cu
+size_t classify_workspace_bytes(const svga_problem *p, int n_rows);
+svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
+                         const int32_t *w_spatial, const int32_t *w_temporal,
+                         const int32_t *rows, int n_rows, float scale, int32_t *head_type_out,
+                         float *mse_out, void *ws, size_t ws_bytes, void *stream);
+
+}  // namespace svga

@@ -1,0 +1,239 @@
+/*
+ * svga.h -- C ABI of the block-sparse spatio-temporal attention library (B200, sm_100a).
+ *
+ * The library computes the forward pass of Sparse-VideoGen-style block-sparse
+ * self-attention for video diffusion, as described in "Accelerating Spatio-Temporal
+ * Attention for Video Diffusion on TPUs" (Google for Developers), of which three
+ * summaries exist: ainews.tenesys.com (Polish), aihirek.info (Hungarian) and
+ * oossa.com (German).  Citations below name the page and its section.
+ *
+ * Conventions for every call:
+ *   - Tensors are DEVICE pointers to contiguous [heads, tokens, head_dim] bf16
+ *     (row-major, head_dim fastest), 16-byte aligned.  tokens = F * H * W.
+ *   - The caller owns all memory.  The library never allocates device memory;
+ *     sizes of the caller-provided buffers come from the *_size queries.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) unless stated otherwise.
+ *   - Arguments are validated on the host before any launch.  A failed check
+ *     returns a status other than SVGA_OK and launches nothing; the message is
+ *     available from svga_last_error() (thread-local).
+ *   - Kernels that wait on the GPU (mbarrier waits) give up after about one
+ *     second, write SVGA_ERR_TIMEOUT into the caller's status word (when one is
+ *     given) and return; the CUDA context stays usable.
+ *   - Launch errors are reported as SVGA_ERR_CUDA.
+ */
+#ifndef SVGA_H
+#define SVGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SVGA_VERSION 1
+
+#if defined(__GNUC__)
+#define SVGA_API __attribute__((visibility("default")))
+#else
+#define SVGA_API
+#endif
+
+typedef void *svga_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    SVGA_OK = 0,
+    SVGA_ERR_INVALID_ARG = 1, /* null pointer, bad enum value, negative band ... */
+    SVGA_ERR_SHAPE = 2,       /* sizes outside the supported range */
+    SVGA_ERR_ALIGNMENT = 3,   /* a pointer not aligned as required */
+    SVGA_ERR_UNSUPPORTED = 4, /* a valid request this build does not implement */
+    SVGA_ERR_WORKSPACE = 5,   /* a caller buffer smaller than the size query says */
+    SVGA_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    SVGA_ERR_TIMEOUT = 7      /* written by a kernel that gave up waiting */
+} svga_status;
+
+/* Head types.  Spatial heads attend to patches of the same or nearby frames;
+ * temporal heads follow a small in-frame region across many frames (aihirek.info,
+ * section "A Sparse VideoGen a figyelmi fejeket osztalyozza"). */
+enum { SVGA_HEAD_SPATIAL = 0, SVGA_HEAD_TEMPORAL = 1 };
+
+/* Token orders.  Tokens arrive frame-major (position f*S + s).  The pages move the
+ * tokens of temporal heads to temporal-major order (ainews.tenesys.com, "Co sie
+ * zmienilo?" item 5) without giving the exact map.  This library's reading:
+ *   SVGA_ORDER_TEMPORAL_MAJOR: frame-0 tokens first (position s), then the other
+ *       frames s-major: position S + s*(F-1) + (f-1)  ("anchor-first");
+ *   SVGA_ORDER_TEMPORAL_MAJOR_STRICT: the literal transpose, position s*F + f. */
+enum {
+    SVGA_ORDER_FRAME_MAJOR = 0,
+    SVGA_ORDER_TEMPORAL_MAJOR = 1,
+    SVGA_ORDER_TEMPORAL_MAJOR_STRICT = 2
+};
+
+/* Flags of svga_sparse_attention_fwd. */
+enum {
+    /* Naive traversal: every visited tile goes through the masked (boundary) path,
+     * the first sparse kernel of the pages, which masked exactly inside every
+     * visited tile (aihirek.info, section "A TPU-kernel kialakitasa dontonek
+     * bizonyult"; ainews.tenesys.com, "Co sie zmienilo?" item 1). */
+    SVGA_FLAG_NAIVE_B1 = 1
+};
+
+/* The problem.  Host struct; the arrays it points to are HOST arrays of `heads`
+ * entries and are read during the call only.
+ *   heads          number of attention heads (1 .. 4096)
+ *   num_frames     F >= 1;  grid_h, grid_w: patch grid, S = grid_h * grid_w
+ *                  tokens N = F * S, 1 <= N <= 2^24, S <= 65535, F <= 65535
+ *   head_dim       64 or 128
+ *   head_type      SVGA_HEAD_SPATIAL or SVGA_HEAD_TEMPORAL per head
+ *   band           per head: spatial keeps |f_q - f_k| <= band (frames); temporal
+ *                  keeps |s_q - s_k| <= band on the flattened in-frame index
+ *                  s = row * grid_w + col.  Inclusive, >= 0.
+ *   order          per head: the token order Q, K, V (and O) of that head are in
+ *   anchor_frame0  1: every query also keeps all keys of frame 0, the anchor
+ *                  (aihirek.info, section "A Sparse VideoGen ..."); 0: no anchor
+ *   tile_q, tile_k tile size of the block map: 64, 128 or 256 each */
+typedef struct {
+    int heads;
+    int num_frames;
+    int grid_h;
+    int grid_w;
+    int head_dim;
+    const int32_t *head_type;
+    const int32_t *band;
+    const int32_t *order;
+    int anchor_frame0;
+    int tile_q;
+    int tile_k;
+} svga_problem;
+
+/* The block map.  DEVICE buffers owned by the caller, sized by svga_block_map_size.
+ *   cls       uint8 [heads][n_q][n_k]: 0 = no kept pair (skipped), 1 = every pair
+ *             kept (full: unmasked fast path), 2 = some kept (boundary: masked).
+ *             Classes are taken on the grid padded to whole tiles, where padded
+ *             pairs count as not kept, so a tile holding padding is never full.
+ *   full_ptr  int32 [heads * n_q + 1]: CSR row pointers over rows r = h * n_q + i
+ *   full_idx  int32 [full_cap]: ascending k-tile indices of the full tiles of row r
+ *             in full_idx[full_ptr[r] .. full_ptr[r+1])
+ *   bnd_ptr, bnd_idx: the same for the boundary tiles
+ *   plan      execution plan of the attention kernel (work items in longest-first
+ *             order and their merged tile lists), plan_bytes long; its layout is
+ *             internal to the library
+ *   status    int32 device word or NULL; cleared by each call that takes the map,
+ *             set to an svga_status by a kernel that fails on the device.
+ * Full/boundary specialisation: full tiles take an unmasked fast path, only
+ * boundary tiles are masked by coordinates (aihirek.info, section "A TPU-kernel
+ * kialakitasa ..."; ainews.tenesys.com, "Co sie zmienilo?" item 2). */
+typedef struct {
+    uint8_t *cls;
+    int32_t *full_ptr;
+    int32_t *full_idx;
+    int32_t *bnd_ptr;
+    int32_t *bnd_idx;
+    int64_t full_cap;
+    int64_t bnd_cap;
+    void *plan;
+    size_t plan_bytes;
+    int32_t *status;
+} svga_block_map;
+
+/* Sizes of the block map buffers and of the build workspace (host-only, no GPU).
+ * Any output pointer may be NULL.  Capacities are worst-case (every tile in a list),
+ * so a map built with them never overflows. */
+SVGA_API svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes,
+                                size_t *ptr_bytes, int64_t *full_cap, int64_t *bnd_cap,
+                                size_t *plan_bytes, size_t *workspace_bytes);
+
+/* Classify every (q-tile, k-tile) pair of every head as empty / full / boundary for
+ * the tokens in order[h], and build the per-q-tile ascending CSR lists of full and
+ * boundary tiles plus the execution plan.  Tile skipping over such lists is the core
+ * of the method (aihirek.info, section "A TPU-kernel kialakitasa ..."; ainews.tenesys.com,
+ * "Co sie zmienilo?" items 1-2).  The map depends on the problem only, not on Q/K/V,
+ * so one map serves every layer and denoising step with the same problem.
+ * workspace: DEVICE buffer of at least the queried size, caller-owned, scratch. */
+SVGA_API svga_status svga_build_block_map(const svga_problem *problem, svga_block_map *map,
+                                 void *workspace, size_t workspace_bytes,
+                                 svga_stream_t stream);
+
+/* Token permutation of one tensor [heads, tokens, head_dim] bf16: for every head h,
+ * dst[h, pos] = src[h, t] where pos is the position of frame-major token t in
+ * order[h] (spatial heads usually stay frame-major: a plain copy).  The pages move
+ * temporal heads to temporal-major order (ainews.tenesys.com, "Co sie zmienilo?"
+ * item 5).  src and dst must not overlap.  Bit-exact copy. */
+SVGA_API svga_status svga_permute_tokens(const void *src, void *dst, const svga_problem *problem,
+                                svga_stream_t stream);
+
+/* Inverse of svga_permute_tokens: dst[h, t] = src[h, pos]. */
+SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svga_problem *problem,
+                                  svga_stream_t stream);
+
+/* Block-sparse attention forward.  For head h and query position i (order[h]):
+ *   O[h,i,:] = sum_{k in K(i)} exp(x_ik - m_i) V[h,k,:] / sum_{k in K(i)} exp(x_ik - m_i)
+ *   x_ik = scale * Q[h,i,:] . K[h,k,:],   m_i = max_{k in K(i)} x_ik,
+ *   lse[h,i] = m_i + ln sum_{k in K(i)} exp(x_ik - m_i)      (natural log)
+ * where K(i) is the set of keys the head's mask keeps, evaluated on the tokens'
+ * original (frame, in-frame index) coordinates.  Skipped tiles hold no kept pair,
+ * full tiles run without mask arithmetic, boundary tiles are masked element by
+ * element (aihirek.info, section "A TPU-kernel kialakitasa ...").  An empty row
+ * gives O = 0 and lse = -inf.
+ *   q, k, v, o : DEVICE bf16 [heads, tokens, head_dim], every head in order[h]
+ *   lse        : DEVICE float [heads, tokens] or NULL
+ *   map        : built by svga_build_block_map for this same problem
+ *   scale      : softmax scale, usually 1/sqrt(head_dim)
+ *   flags      : 0 or SVGA_FLAG_NAIVE_B1
+ * bf16 inputs, fp32 accumulation and softmax, P rounded to bf16 for the PV product. */
+SVGA_API svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                                      float *lse, const svga_problem *problem,
+                                      const svga_block_map *map, float scale, int flags,
+                                      svga_stream_t stream);
+
+/* Dense attention forward (every pair kept): the same-GPU dense baseline, the role
+ * dense Splash Attention plays on the pages (aihirek.info, section "A TPU-kernel
+ * kialakitasa ..."; oossa.com, "Die Fakten").  Same kernel, every tile unmasked
+ * except the ragged last key tile, which is length-masked.
+ *   status: DEVICE int32 word or NULL (cleared, then set on a device failure). */
+SVGA_API svga_status svga_dense_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                                     float *lse, int heads, int tokens, int head_dim,
+                                     float scale, int32_t *status, svga_stream_t stream);
+
+/* Workspace for svga_classify_heads with n_rows sampled query rows per head. */
+SVGA_API svga_status svga_classify_size(const svga_problem *problem, int n_rows,
+                               size_t *workspace_bytes);
+
+/* Online head classification.  For a few query rows per head, compute the dense
+ * output and the outputs under the spatial and the temporal mask, and give the head
+ * the mask whose output deviates least from the dense one (aihirek.info, section
+ * "A Sparse VideoGen a figyelmi fejeket osztalyozza").  Deviation = mean squared
+ * error over the sampled rows x head_dim; a tie goes to spatial.
+ *   q, k, v     : DEVICE bf16 [heads, tokens, head_dim] in FRAME-MAJOR order
+ *   problem     : shape, anchor and head_dim; head_type/band/order are not read
+ *   w_spatial   : HOST int32 [heads], spatial band of the candidate mask
+ *   w_temporal  : HOST int32 [heads], temporal band of the candidate mask
+ *   rows        : DEVICE int32 [n_rows] frame-major token indices shared by all
+ *                 heads, or NULL for the default rule r_i = floor((2i+1) N / (2 n_rows))
+ *   n_rows      : sampled rows per head, 1 .. N
+ *   scale       : softmax scale, usually 1/sqrt(head_dim)
+ *   head_type_out : HOST int32 [heads] (written before the call returns)
+ *   mse_out     : HOST float [heads][2] (spatial, temporal) or NULL
+ *   workspace   : DEVICE scratch of at least svga_classify_size bytes
+ * This call synchronises `stream` to return the types to the host. */
+SVGA_API svga_status svga_classify_heads(const void *q, const void *k, const void *v,
+                                const svga_problem *problem, const int32_t *w_spatial,
+                                const int32_t *w_temporal, const int32_t *rows, int n_rows,
+                                float scale, int32_t *head_type_out, float *mse_out, void *workspace,
+                                size_t workspace_bytes, svga_stream_t stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+SVGA_API const char *svga_last_error(void);
+
+/* Name of a status code. */
+SVGA_API const char *svga_status_string(svga_status status);
+
+/* SVGA_VERSION of the built library. */
+SVGA_API int svga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVGA_H */

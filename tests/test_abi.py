@@ -1,0 +1,113 @@
+"""The C-ABI library: loads without a GPU, exports every symbol the header declares, and
+rejects bad arguments on the host before any launch (CPU only: no compute call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_spatio_attn_b200 import configs as C
+from block_sparse_spatio_attn_b200 import svga
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "svga.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svga_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_spatio_attn_b200 import build
+    build.build()
+    return svga.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+    assert set(names) == set(svga.EXPORTED)
+
+
+def test_version_and_status_strings(lib):
+    assert svga.version() == 1
+    assert svga.status_string(0) == "SVGA_OK"
+    assert svga.status_string(7) == "SVGA_ERR_TIMEOUT"
+
+
+def test_block_map_sizes_headline(lib):
+    wl = C.headline()
+    s = svga.svga_block_map_size(svga.ProblemSpec.from_workload(wl))
+    nq = -(-75600 // 128)
+    assert s["cls_bytes"] == 10 * nq * nq
+    assert s["ptr_bytes"] == 4 * (10 * nq + 1)
+    assert s["full_cap"] == s["bnd_cap"] == 10 * nq * nq
+    n_items = 10 * ((nq + 1) // 2)
+    hdr = (64 + 16 * (10 + n_items) + 255) // 256 * 256
+    assert s["plan_bytes"] == hdr + 4 * n_items * nq
+
+
+def _bad(lib, **kw):
+    wl = C.tiny()
+    d = dict(heads=wl.heads, num_frames=wl.frames, grid_h=wl.grid_h, grid_w=wl.grid_w,
+             head_dim=wl.head_dim, head_type=wl.head_type, band=wl.band, order=wl.order,
+             anchor_frame0=1, tile_q=64, tile_k=64)
+    d.update(kw)
+    return svga.ProblemSpec(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(heads=0, head_type=[], band=[], order=[]), 2),
+    (dict(head_dim=96), 4),
+    (dict(tile_q=32), 4),
+    (dict(tile_k=512), 4),
+    (dict(band=[-1, 8]), 1),
+    (dict(head_type=[0, 5]), 1),
+    (dict(order=[0, 3]), 1),
+    (dict(anchor_frame0=2), 1),
+    (dict(num_frames=0), 2),
+    (dict(grid_h=300, grid_w=300), 2),
+])
+def test_problem_validation(lib, kw, status):
+    with pytest.raises(svga.SvgaError) as e:
+        svga.svga_block_map_size(_bad(lib, **kw))
+    assert e.value.status == status
+
+
+def test_pointer_validation_before_launch(lib):
+    prob = _bad(lib)
+    P = ctypes.c_void_p
+    st = P(0)
+    # NULL and misaligned tensors are rejected on the host, before any CUDA call
+    rc = lib.svga_permute_tokens(None, P(4096), ctypes.byref(prob.c), st)
+    assert rc == 1
+    rc = lib.svga_permute_tokens(P(4096 + 8), P(1 << 20), ctypes.byref(prob.c), st)
+    assert rc == 3
+    rc = lib.svga_permute_tokens(P(4096), P(4096 + 256), ctypes.byref(prob.c), st)
+    assert rc == 1 and b"overlap" in lib.svga_last_error()
+    rc = lib.svga_dense_attention_fwd(P(4096), P(4096), P(4096), P(4096), None, 2, 192, 80,
+                                      ctypes.c_float(0.1), None, st)
+    assert rc == 4
+    rc = lib.svga_dense_attention_fwd(P(4096), P(4096), P(4096), P(4096), None, 2, 192, 64,
+                                      ctypes.c_float(-1.0), None, st)
+    assert rc == 1
+    m = svga.BlockMapC()
+    rc = lib.svga_sparse_attention_fwd(P(4096), P(4096), P(4096), P(4096), None,
+                                       ctypes.byref(prob.c), ctypes.byref(m),
+                                       ctypes.c_float(0.1), 0, st)
+    assert rc == 1
+    rc = lib.svga_build_block_map(ctypes.byref(prob.c), ctypes.byref(m), None, 0, st)
+    assert rc == 1
+
+
+def test_classify_size_validation(lib):
+    prob = svga.ProblemSpec.from_workload(C.tiny())
+    assert svga.svga_classify_size(prob, 2) > 0
+    with pytest.raises(svga.SvgaError):
+        svga.svga_classify_size(prob, 0)
+    with pytest.raises(svga.SvgaError):
+        svga.svga_classify_size(prob, 193)

@@ -1,0 +1,168 @@
+"""Block-sparse and dense attention on the GPU (through the C ABI) against the fp64 oracle.
+
+Tolerance (bf16 inputs, fp32 accumulation): max-abs 2e-2, relative Frobenius 1e-2,
+LSE max-abs 1e-3.  Full-size workloads are checked on sampled rows, including whole
+128-row blocks and the ragged last block."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_spatio_attn_b200 import configs as C
+from block_sparse_spatio_attn_b200.inputs import make_qkv
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from block_sparse_spatio_attn_b200 import svga  # noqa: E402
+from tests.helpers import (assert_attn_close, lse_to_frame_major, oracle_rows,  # noqa: E402
+                           run_sparse_path, sample_rows)
+
+_cache = {}
+
+
+def inputs(wl):
+    key = (wl.name, wl.seed, wl.heads)
+    if key not in _cache:
+        q, k, v = make_qkv(wl)
+        _cache.clear()
+        _cache[key] = (q, k, v, q.cuda(), k.cuda(), v.cuda())
+    return _cache[key]
+
+
+def check_sparse(wl, rows=None, naive=False, order=None, tile_q=None, tile_k=None):
+    q, k, v, qd, kd, vd = inputs(wl)
+    order = wl.order if order is None else order
+    o, lse, _ = run_sparse_path(wl, qd, kd, vd, naive=naive, order=order, tile_q=tile_q,
+                                tile_k=tile_k)
+    o = o.float().cpu().numpy()
+    lse = lse_to_frame_major(lse.cpu().numpy(), wl, order)
+    rows = np.arange(wl.tokens, dtype=np.int32) if rows is None else rows
+    for h in range(wl.heads):
+        ro, rl = oracle_rows(wl, q, k, v, h, rows)
+        assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"{wl.name} head {h}")
+
+
+def test_tiny_sparse_all_rows():
+    check_sparse(C.tiny())
+
+
+def test_tiny_sparse_naive_b1():
+    check_sparse(C.tiny(), naive=True)
+
+
+def test_tiny_temporal_major_orders():
+    check_sparse(C.tiny(), order=[C.ORDER_TEMPORAL_MAJOR, C.ORDER_TEMPORAL_MAJOR])
+    check_sparse(C.tiny(), order=[C.ORDER_TEMPORAL_MAJOR_STRICT] * 2)
+
+
+def test_mid_sparse():
+    wl = C.mid()
+    check_sparse(wl, rows=sample_rows(wl, 600))
+
+
+def test_mid_sparse_naive_b1_equals_b2():
+    wl = C.mid()
+    q, k, v, qd, kd, vd = inputs(wl)
+    o1, l1, _ = run_sparse_path(wl, qd, kd, vd, naive=False)
+    o2, l2, _ = run_sparse_path(wl, qd, kd, vd, naive=True)
+    # the same arithmetic in the same order: masking only removes pairs that are kept
+    # anyway on full tiles, so the results agree to the last bit
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("tq,tk", [(64, 64), (256, 128), (128, 256), (256, 256), (64, 128)])
+def test_mid_tile_sizes(tq, tk):
+    wl = C.mid()
+    check_sparse(wl, rows=sample_rows(wl, 200, seed=tq + tk), tile_q=tq, tile_k=tk)
+
+
+def test_mid_frame_major_temporal():
+    wl = C.mid()
+    check_sparse(wl, rows=sample_rows(wl, 200, seed=3), order=[C.ORDER_FRAME_MAJOR] * 4)
+
+
+def test_headline_sparse_sampled():
+    wl = C.headline()
+    check_sparse(wl, rows=sample_rows(wl, 160))
+
+
+def test_permstudy_strict_order_sampled():
+    wl = C.permutation_study(C.ORDER_TEMPORAL_MAJOR_STRICT)
+    check_sparse(wl.__class__(**{**wl.__dict__, "head_type": wl.head_type[:2],
+                                 "band": wl.band[:2], "order": wl.order[:2]}),
+                 rows=sample_rows(wl, 120))
+
+
+def dense_check(wl, rows):
+    q, k, v, qd, kd, vd = inputs(wl)
+    o = torch.empty_like(qd)
+    lse = torch.empty(wl.heads, wl.tokens, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    svga.svga_dense_attention_fwd(qd, kd, vd, o, lse, 1.0 / math.sqrt(wl.head_dim), st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    for h in range(wl.heads):
+        ro, rl = oracle_rows(wl, q, k, v, h, rows, type_=oracle.DENSE, band=0)
+        assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"dense {wl.name} head {h}")
+
+
+def test_tiny_dense_all_rows():
+    wl = C.tiny()
+    dense_check(wl, np.arange(wl.tokens, dtype=np.int32))
+
+
+def test_mid_dense_sampled():
+    wl = C.mid()
+    dense_check(wl, sample_rows(wl, 300))
+
+
+def test_headline_dense_sampled():
+    wl = C.headline()
+    wl2 = wl.__class__(**{**wl.__dict__, "head_type": wl.head_type[:3], "band": wl.band[:3],
+                          "order": wl.order[:3]})
+    dense_check(wl2, sample_rows(wl2, 96))
+
+
+@pytest.mark.parametrize("N_frames,gh,gw,d", [(2, 5, 10, 128), (1, 7, 9, 64), (3, 1, 43, 128)])
+def test_small_and_ragged_shapes(N_frames, gh, gw, d):
+    """One block, an odd number of blocks, single frame, N < 128."""
+    wl = C.Workload("odd", N_frames, gh, gw, d, [C.SPATIAL, C.TEMPORAL], [0, 3],
+                    [C.ORDER_FRAME_MAJOR, C.ORDER_TEMPORAL_MAJOR], seed=9)
+    check_sparse(wl)
+    dense_check(wl, np.arange(wl.tokens, dtype=np.int32))
+
+
+def test_special_values():
+    """V constant -> O equals it; Q = 0 -> plain masked mean of V (via the oracle)."""
+    wl = C.mid()
+    q, k, v, qd, kd, vd = inputs(wl)
+    c = torch.linspace(-1, 1, wl.head_dim).to(torch.bfloat16)
+    vc = c.expand(wl.heads, wl.tokens, wl.head_dim).contiguous().cuda()
+    o, _, _ = run_sparse_path(wl, qd, kd, vc)
+    err = (o.float().cpu() - c.float()).abs().max().item()
+    assert err <= 1e-2
+    qz = torch.zeros_like(qd)
+    o, lse, _ = run_sparse_path(wl, qz, kd, vd)
+    rows = sample_rows(wl, 100, seed=5)
+    o = o.float().cpu().numpy()
+    lse = lse_to_frame_major(lse.cpu().numpy(), wl, wl.order)
+    zq = torch.zeros_like(q)
+    for h in range(wl.heads):
+        ro, rl = oracle_rows(wl, zq, k, v, h, rows)
+        assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"Q=0 head {h}")
+
+
+def test_repeatable_bitwise():
+    wl = C.mid()
+    q, k, v, qd, kd, vd = inputs(wl)
+    o1, l1, _ = run_sparse_path(wl, qd, kd, vd)
+    o2, l2, _ = run_sparse_path(wl, qd, kd, vd)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
