@@ -26,7 +26,7 @@ _cache = {}
 
 
 def inputs(wl):
-    key = (wl.name, wl.seed, wl.heads)
+    key = (wl.name, wl.seed, wl.heads, wl.frames, wl.grid_h, wl.grid_w, wl.head_dim)
     if key not in _cache:
         q, k, v = make_qkv(wl)
         _cache.clear()
