@@ -1,0 +1,435 @@
+"""Benchmark of the block-sparse spatio-temporal attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl svga|reference]
+                    [--config headline|mid|tiny|permstudy|2k] [--tile 128x128]
+
+One step = one pass of the hot path over the workload's Q/K/V already in HBM:
+token permutation of Q, K, V into each head's order, block-sparse attention, inverse
+permutation of O.  The block map depends on the problem only and is built once before
+timing (its build time is reported separately), as it would be cached across layers and
+denoising steps.  Metric: effective TFLOP/s on kept pairs, FLOP = sum over heads of
+4 * kept_pairs * head_dim, and ms per step.  Under torchrun every rank runs the same
+workload on its own GPU (weak scaling); value = FLOP of all ranks / max time over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this method has) on a
+bounded sample of query rows per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_spatio_attn_b200 import configs as C  # noqa: E402
+from block_sparse_spatio_attn_b200.inputs import make_qkv  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "sparse attn fwd ms + TFLOP/s on kept pairs (75.6K tok, 10 heads, d=128)"
+
+
+# ------------------------------------------------------------------- accounting
+def kept_pairs(type_: int, band: int, anchor: int, F: int, S: int) -> int:
+    """Kept (q, k) pairs of one head (closed form of the spatial / temporal masks)."""
+    if type_ == C.SPATIAL:
+        tot = 0
+        for fq in range(F):
+            lo, hi = max(0, fq - band), min(F - 1, fq + band)
+            tot += (hi - lo + 1) + (1 if (anchor and lo > 0) else 0)
+        return S * S * tot
+    c = sum(min(S - 1, s + band) - max(0, s - band) + 1 for s in range(S))
+    return F * S * S + F * (F - 1) * c if anchor else F * F * c
+
+
+def kept_keys_of_row(wl, h: int, t: int) -> int:
+    """Kept keys of frame-major query token t of head h."""
+    F, S = wl.frames, wl.tokens_per_frame
+    f, s = divmod(t, S)
+    w = wl.band[h]
+    if wl.head_type[h] == C.SPATIAL:
+        lo, hi = max(0, f - w), min(F - 1, f + w)
+        return S * ((hi - lo + 1) + (1 if (wl.anchor_frame0 and lo > 0) else 0))
+    c = min(S - 1, s + w) - max(0, s - w) + 1
+    return S + (F - 1) * c if wl.anchor_frame0 else F * c
+
+
+def kept_flops(wl) -> float:
+    F, S, d = wl.frames, wl.tokens_per_frame, wl.head_dim
+    return float(sum(4 * kept_pairs(t, w, wl.anchor_frame0, F, S) * d
+                     for t, w in zip(wl.head_type, wl.band)))
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def traffic_from_profile(kernel_src: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it
+    was taken on the current kernel source (sha256 recorded in the summary)."""
+    path = os.path.join(ROOT, "profiles", "attention_headline_ncu.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt)
+    if not (m_sha and m_b):
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return float(m_b.group(1)) if sha == m_sha.group(1) else None
+
+
+# ------------------------------------------------------------------ clock sampler
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self, gpu_index: int):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((int(parts[0]), float(parts[1]), float(parts[2]),
+                                 float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0,
+                                 parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.f.name)
+        idx = {r[0] for r in rows}
+        gi = gpu_index if gpu_index in idx else (min(idx) if idx else None)
+        rows = [r for r in rows if r[0] == gi]
+        if not rows:
+            return None
+        load = [r for r in rows if r[3] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[4]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in load), "sm_max_mhz": rows[0][2],
+                "reasons": reasons, "samples": len(load)}
+
+
+# --------------------------------------------------------------------- svga arm
+def run_svga(args, rank, world, local_rank):
+    from block_sparse_spatio_attn_b200 import svga
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = C.ALL[args.config]()
+    if args.tile:
+        tq, tk = (int(x) for x in args.tile.lower().split("x"))
+        wl = wl.with_tile(tq, tk)
+    H, N, d = wl.heads, wl.tokens, wl.head_dim
+    scale = 1.0 / math.sqrt(d)
+    q, k, v = make_qkv(wl)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    prob = svga.ProblemSpec.from_workload(wl)
+    stream = torch.cuda.current_stream(dev)
+
+    # block map: built once (timed on its own)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bmap = svga.build_block_map(prob)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(3):
+        svga.svga_build_block_map(prob, bmap)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    map_ms = ev0.elapsed_time(ev1) / 3
+    nq, nk = -(-N // wl.tile_q), -(-N // wl.tile_k)
+    cls = bmap.cls[: H * nq * nk].view(H, nq, nk).cpu()
+    visited = int((cls != 0).sum())
+    boundary = int((cls == 2).sum())
+    visited_flops = 4.0 * wl.tile_q * wl.tile_k * d * visited
+    kflops = kept_flops(wl)
+    kept_frac = kflops / (4.0 * H * N * N * d)
+
+    qp, kp, vp, op, o = (torch.empty_like(qd) for _ in range(5))
+
+    def step(attn_evs=None):
+        svga.svga_permute_tokens(qd, qp, prob)
+        svga.svga_permute_tokens(kd, kp, prob)
+        svga.svga_permute_tokens(vd, vp, prob)
+        if attn_evs is not None:
+            attn_evs[0].record(stream)
+        svga.svga_sparse_attention_fwd(qp, kp, vp, op, None, prob, bmap, scale)
+        if attn_evs is not None:
+            attn_evs[1].record(stream)
+        svga.svga_unpermute_tokens(op, o, prob)
+
+    launches_per_step = 5
+    if args.mode == "attn":
+        # profiling aid: the attention kernel alone, warm-up + steps launches, no report
+        step()
+        for _ in range(args.warmup + args.steps):
+            svga.svga_sparse_attention_fwd(qp, kp, vp, op, None, prob, bmap, scale)
+        torch.cuda.synchronize()
+        if bmap.device_status() != 0:
+            raise RuntimeError(f"device status {bmap.device_status()}")
+        return None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if bmap.device_status() != 0:
+        raise RuntimeError(f"device status {bmap.device_status()} after warm-up")
+
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    attn_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(attn_evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(local_rank) if rank == 0 else None
+    elapsed = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_evs)
+    if world > 1:
+        t = torch.tensor([elapsed, attn_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed, attn_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed / args.steps
+    if bmap.device_status() != 0:
+        raise RuntimeError(f"device status {bmap.device_status()} in the timed region")
+
+    # -------- extras on the same GPU (not part of `value`) ------------------------
+    def time_it(fn, reps):
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    reps = max(3, min(args.steps, 10))
+    dense_ms = time_it(lambda: svga.svga_dense_attention_fwd(qd, kd, vd, op, None, scale), reps)
+    naive_ms = time_it(lambda: svga.svga_sparse_attention_fwd(qp, kp, vp, op, None, prob, bmap,
+                                                              scale, svga.FLAG_NAIVE_B1), reps)
+    perm_ms = time_it(lambda: svga.svga_permute_tokens(qd, qp, prob), reps)
+    dense_flops = 4.0 * H * N * N * d
+
+    # -------- end to end through the public API, host buffers ---------------------
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(q).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+
+    peaks, peak_src = read_peaks()
+    timed_s = elapsed / 1e3
+    sustained = timed_s >= 2.0
+    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    achieved = visited_flops / (attn_ms * 1e-3) / 1e12
+    traffic = traffic_from_profile(os.path.join(ROOT, "block_sparse_spatio_attn_b200", "csrc",
+                                                "attention.cu"))
+    if traffic is not None and args.config != "headline":
+        traffic = None
+    total_flops = kflops * world
+    out = {
+        "metric": METRIC, "value": total_flops / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": N, "heads": H, "head_dim": d,
+                   "frames": wl.frames, "grid": f"{wl.grid_h}x{wl.grid_w}",
+                   "head_types": "".join("ST"[t] for t in wl.head_type), "bands": wl.band,
+                   "orders": wl.order, "tile": f"{wl.tile_q}x{wl.tile_k}",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (Q,K,V %.0f MB)" % (3 * H * N * d * 2 / 1e6),
+                   "step": "permute QKV + sparse attention + unpermute O"},
+        "attn_ms": attn_ms,
+        "attn_tflops_kept": kflops / (attn_ms * 1e-3) / 1e12,
+        "attn_tflops_visited": achieved,
+        "kept_fraction": kept_frac, "visited_fraction": visited / (H * nq * nk),
+        "boundary_fraction": boundary / (H * nq * nk),
+        "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+        "sparse_over_dense": attn_ms / dense_ms, "target_ratio": kept_frac + 0.15,
+        "naive_b1_ms": naive_ms, "permute_ms_per_tensor": perm_ms, "map_build_ms": map_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} {'sustained' if sustained else 'burst'} bf16",
+                     "kernel": "attn_fwd_kernel<128,128>", "flops_per_launch": visited_flops},
+        "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * H * N * d * 2,
+                "d2h_bytes_per_step": H * N * d * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, q, k, v, args.cpu_seconds)
+    return out
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(wl, q, k, v, rows_per_head: int, seed: int):
+    """Run the oracle on `rows_per_head` rows of every head; returns (seconds, kept FLOP)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    N = wl.tokens
+    rows = np.sort(rng.choice(N, size=rows_per_head, replace=False)).astype(np.int32)
+    t = time.perf_counter()
+    flops = 0.0
+    for h in range(wl.heads):
+        oracle.attention_rows(q[h].float().numpy(), k[h].float().numpy(), v[h].float().numpy(),
+                              wl.frames, wl.tokens_per_frame, 1.0 / math.sqrt(wl.head_dim),
+                              wl.head_type[h], wl.band[h], wl.anchor_frame0, rows)
+        flops += sum(4.0 * kept_keys_of_row(wl, h, int(r)) * wl.head_dim for r in rows)
+    return time.perf_counter() - t, flops
+
+
+def calibrate_rows(wl, q, k, v, seconds: float) -> int:
+    dt, _ = oracle_sample(wl, q, k, v, 8, 123)
+    return max(8, min(wl.tokens, int(8 * seconds / max(dt, 1e-3))))
+
+
+def cpu_baseline(wl, q, k, v, seconds: float):
+    import oracle
+    rows = calibrate_rows(wl, q, k, v, seconds)
+    dt, fl = oracle_sample(wl, q, k, v, rows, 7)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} query rows per head x {wl.heads} heads of {wl.name} "
+                      f"(fp64 C + OpenMP), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    import oracle
+    if rank != 0:
+        return None
+    wl = C.ALL[args.config]()
+    q, k, v = make_qkv(wl)
+    rows = calibrate_rows(wl, q, k, v, args.ref_step_seconds)
+    for i in range(args.warmup):
+        oracle_sample(wl, q, k, v, rows, 1000 + i)
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl = oracle_sample(wl, q, k, v, rows, i)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = f"{rows} query rows per head x {wl.heads} heads per step of {wl.name}"
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "tokens": wl.tokens, "heads": wl.heads,
+                       "head_dim": wl.head_dim, "tile": f"{wl.tile_q}x{wl.tile_k}"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="svga", choices=["svga", "reference"])
+    ap.add_argument("--config", default="headline", choices=sorted(C.ALL))
+    ap.add_argument("--tile", default="")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="full", choices=["full", "attn"],
+                    help="attn: only launch the attention kernel (for ncu captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = world > 1 and args.impl == "svga"   # the oracle arm runs on rank 0 alone
+    if pg:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, rank, world)
+        else:
+            out = run_svga(args, rank, world, local_rank)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if pg:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
