@@ -24,7 +24,8 @@ HEAD_SPATIAL, HEAD_TEMPORAL = 0, 1
 ORDER_FRAME_MAJOR, ORDER_TEMPORAL_MAJOR, ORDER_TEMPORAL_MAJOR_STRICT = 0, 1, 2
 FLAG_NAIVE_B1 = 1
 
-EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_permute_tokens",
+EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",
+            "svga_permute_tokens",
             "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_dense_attention_fwd",
             "svga_classify_size", "svga_classify_heads", "svga_last_error",
             "svga_status_string", "svga_version"]
@@ -73,6 +74,7 @@ def load() -> ctypes.CDLL:
                                             ctypes.POINTER(ctypes.c_int64),
                                             ctypes.POINTER(SZ), ctypes.POINTER(SZ)]
         lib.svga_build_block_map.argtypes = [PP, ctypes.POINTER(BlockMapC), P, SZ, P]
+        lib.svga_build_block_map_static.argtypes = [PP, ctypes.POINTER(BlockMapC), P]
         lib.svga_permute_tokens.argtypes = [P, P, PP, P]
         lib.svga_unpermute_tokens.argtypes = [P, P, PP, P]
         lib.svga_sparse_attention_fwd.argtypes = [P, P, P, P, P, PP, ctypes.POINTER(BlockMapC),

@@ -155,6 +155,27 @@ SVGA_API svga_status svga_build_block_map(const svga_problem *problem, svga_bloc
                                  void *workspace, size_t workspace_bytes,
                                  svga_stream_t stream);
 
+/* Size of the library's static build scratch used by svga_build_block_map_static. */
+#define SVGA_MAP_STATIC_SCRATCH_BYTES (1u << 20)
+
+/* svga_build_block_map without a workspace argument, for callers that cannot allocate
+ * device memory when they build a map: plugin hosts whose execute callback forbids
+ * allocation, servers that fix their memory budget at start-up, code that must not take
+ * the implicit device synchronisation of cudaMalloc / cudaFree.  The paper has no
+ * counterpart; it is a deployment convenience.
+ *   - The caller still provides every output buffer of `map` (svga_block_map_size).
+ *   - The build's scratch lives in one static device array of
+ *     SVGA_MAP_STATIC_SCRATCH_BYTES that each GPU loading the library keeps until the
+ *     process exits.  A problem needing more scratch (svga_block_map_size's
+ *     workspace_bytes) is rejected with SVGA_ERR_WORKSPACE and nothing is launched.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - The call allocates nothing.  All calls share the array: calls that overlap on the
+ *     GPU (unordered streams) race; calls ordered on one stream are safe.
+ * Results are identical to svga_build_block_map's. */
+SVGA_API svga_status svga_build_block_map_static(const svga_problem *problem,
+                                                 svga_block_map *map, svga_stream_t stream);
+
 /* Token permutation of one tensor [heads, tokens, head_dim] bf16: for every head h,
  * dst[h, pos] = src[h, t] where pos is the position of frame-major token t in
  * order[h] (spatial heads usually stay frame-major: a plain copy).  The pages move
