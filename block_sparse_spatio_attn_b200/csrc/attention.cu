@@ -16,10 +16,15 @@
 //       O_i += P_i V   (A = P from TMEM as bf16, B = V from shared memory)
 //     in the order S0(n+1) after PV0(n) and S1(n+1) after PV1(n), so the two softmax
 //     warpgroups work on different tiles while the tensor core runs the other's MMAs;
+//     operand descriptors are built once and advanced by constant offsets;
 //   * warps 4-7 and 8-11 hold one query row per thread (TMEM lane = row): they read S,
-//     apply the mask on boundary tiles, run the online softmax in the exp2 domain,
-//     write P back into TMEM over S, and rescale O in TMEM only when the running
-//     maximum grows by more than 2^8 (P stays <= 256 otherwise);
+//     run the online softmax in the exp2 domain with packed fp32x2 arithmetic (part of
+//     the exponentials on the FMA pipe by polynomial, the rest on the MUFU unit), write
+//     P back into TMEM over S, and rescale O in TMEM only when the running maximum grows
+//     by more than 2^8 (P stays <= 256 otherwise);
+//   * boundary tiles build a 128-bit keep mask per row from the runs of the key chunk
+//     (at most a few intervals per run), then mask with one select per element;
+//   * the producer/MMA warpgroup gives registers to the softmax warpgroups (setmaxnreg);
 //   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated).
 //
 // Every mbarrier wait gives up after about a second: the CTA raises a shared abort
@@ -30,9 +35,14 @@
 
 #include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "svga_device.cuh"
 #include "svga_internal.h"
+
+#ifndef SVGA_POLY_EVERY
+#define SVGA_POLY_EVERY 0  // one pair of exponentials in this many on the FMA pipe (0: none)
+#endif
 
 namespace svga {
 namespace {
@@ -40,6 +50,12 @@ namespace {
 constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kNegInfBits = 0xff800000u;
+// Register split: the producer / MMA warpgroup drops to kRegsLow, the two softmax
+// warpgroups rise to kRegsHigh.  128 * kRegsLow + 256 * kRegsHigh must not exceed the
+// 384 * kRegsLaunch registers the CTA is launched with (checked on the host).
+constexpr int kRegsLaunch = 168, kRegsLow = 120, kRegsHigh = 192;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 struct KParams {
     int heads, nq_rows, nk_rows, F, S, anchor;
@@ -66,6 +82,7 @@ struct Cfg {
     static constexpr int kSmemAlloc = kSmemData + kSmemBar + 1024;  // + alignment slack
     static constexpr int kSmemLaunch = kSmemAlloc < 120 * 1024 ? 120 * 1024 : kSmemAlloc;
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+    static_assert((kStages & (kStages - 1)) == 0, "stage count is a power of two");
 };
 
 struct Barriers {
@@ -100,12 +117,13 @@ struct Item {
     }
 };
 
-__device__ __forceinline__ Item make_item(const KParams &p)
+__device__ __forceinline__ Item make_item(const KParams &p, int kn)
 {
     Item it;
     it.mode = p.mode;
     it.naive = p.naive;
     it.n_kc = p.n_kc;
+    it.ragged = (p.nk_rows % kn) != 0;
     if (p.mode == 0) {
         const int4 x = __ldg(p.items + blockIdx.x);
         it.h = x.x;
@@ -122,30 +140,114 @@ __device__ __forceinline__ Item make_item(const KParams &p)
     return it;
 }
 
-// Advance (f, s) to the next position of `order`.
-__device__ __forceinline__ void step_coord(int order, int F, int S, int &f, int &s)
+// Set bits [c0, c1) of a mask of NW 32-bit words (0 <= c0 < c1 <= 32 * NW).
+template <int NW>
+__device__ __forceinline__ void mask_set(uint32_t (&m)[NW], int c0, int c1)
 {
-    if (order == ORDER_FM) {
-        if (++s == S) {
-            s = 0;
-            ++f;
-        }
-    } else if (order == ORDER_TM_STRICT) {
-        if (++f == F) {
-            f = 0;
-            ++s;
-        }
-    } else {
-        if (f == 0) {
-            if (++s == S) {
-                s = 0;
-                f = 1;
-            }
-        } else if (++f == F) {
-            f = 1;
-            ++s;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int lo = max(c0 - 32 * w, 0), hi = min(c1 - 32 * w, 32);
+        if (lo < hi) {
+            const uint32_t upto = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+            m[w] |= upto & ~((1u << lo) - 1u);
         }
     }
+}
+
+// Keep mask of the key positions [k0, k0 + KN) for one query (fq, sq): bit c is set
+// when key k0 + c exists and the head's mask keeps it.  The positions of a chunk are
+// walked row by row of the order's grid (a frame in frame-major order, an in-frame
+// index in the temporal-major orders); in each row the kept keys form at most two
+// intervals, so the mask costs a handful of integer operations per row.
+template <int KN>
+__device__ __forceinline__ void keep_mask(int order, int type, int band, int anchor, int F, int S,
+                                          int N, int fq, int sq, int k0, uint32_t (&m)[KN / 32])
+{
+#pragma unroll
+    for (int w = 0; w < KN / 32; ++w) m[w] = 0u;
+    const int kend = min(k0 + KN, N);
+    int pos = k0, fixed, row_start, row_len, fbase;
+    bool f_fixed;
+    if (order == ORDER_FM) {
+        fixed = pos / S;
+        row_start = fixed * S;
+        row_len = S;
+        f_fixed = true;
+        fbase = 0;
+    } else if (order == ORDER_TM_STRICT) {
+        fixed = pos / F;
+        row_start = fixed * F;
+        row_len = F;
+        f_fixed = false;
+        fbase = 0;
+    } else if (pos < S) {
+        fixed = 0;
+        row_start = 0;
+        row_len = S;
+        f_fixed = true;
+        fbase = 0;
+    } else {
+        fixed = (pos - S) / (F - 1);
+        row_start = S + fixed * (F - 1);
+        row_len = F - 1;
+        f_fixed = false;
+        fbase = 1;
+    }
+    // kept intervals are merged while they touch, so runs of fully kept rows cost one
+    // mask_set
+    int plo = 0, phi = 0;
+    auto flush = [&]() {
+        if (plo < phi) mask_set<KN / 32>(m, plo - k0, phi - k0);
+        plo = phi = 0;
+    };
+#pragma unroll 1
+    while (pos < kend) {
+        const int b = min(kend, row_start + row_len);
+        auto add = [&](int lo, int hi) {
+            lo = max(lo, pos);
+            hi = min(hi, b);
+            if (lo >= hi) return;
+            if (plo < phi && lo == phi) {
+                phi = hi;
+            } else {
+                flush();
+                plo = lo;
+                phi = hi;
+            }
+        };
+        if (type == MASK_DENSE) {
+            add(pos, b);
+        } else if (f_fixed) {  // one frame: s runs along the row
+            const int ff = fixed;
+            if ((anchor && ff == 0) || (type == MASK_SPATIAL && abs(fq - ff) <= band))
+                add(pos, b);
+            else if (type == MASK_TEMPORAL)
+                add(row_start + sq - band, row_start + sq + band + 1);
+        } else {  // one in-frame index: f runs along the row from fbase
+            const int sf = fixed;
+            if (type == MASK_TEMPORAL) {
+                if (abs(sq - sf) <= band)
+                    add(pos, b);
+                else if (anchor && fbase == 0)
+                    add(row_start, row_start + 1);
+            } else {
+                add(row_start + (fq - band) - fbase, row_start + (fq + band) - fbase + 1);
+                if (anchor && fbase == 0) add(row_start, row_start + 1);
+            }
+        }
+        pos = b;
+        if (order == ORDER_TM && f_fixed) {  // leave the frame-0 block
+            f_fixed = false;
+            fbase = 1;
+            fixed = 0;
+            row_start = S;
+            row_len = F - 1;
+        } else {
+            ++fixed;
+            row_start += row_len;
+        }
+    }
+    flush();
 }
 
 template <int D, int KN, bool OUT_F32>
@@ -163,8 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    Item it = make_item(p);
-    it.ragged = (p.nk_rows % KN) != 0;
+    const Item it = make_item(p, KN);
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bar->q_full), 1);
@@ -174,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&bar->s_full[i]), 1);
-            mbar_init(smem_u32(&bar->p_full[i]), 128);
+            mbar_init(smem_u32(&bar->p_full[i]), 4);  // one arrival per softmax warp
             mbar_init(smem_u32(&bar->o_done[i]), 1);
         }
         mbar_init(smem_u32(&bar->drain), 1);
@@ -190,9 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp < 4) {
+        setmaxnreg_dec<kRegsLow>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- TMA producer
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
@@ -207,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int n = 0; n < it.E && ok; ++n) {
                 const int kc = (int)(it.entry(n) & kEntChunkMask);
                 for (int t = 0; t < 2; ++t) {
-                    const int idx = 2 * n + t, s = idx % C::kStages, round = idx / C::kStages;
+                    const int idx = 2 * n + t, s = idx & (C::kStages - 1), round = idx / C::kStages;
                     if (round > 0 &&
                         !mbar_wait(smem_u32(&bar->kv_empty[s]), (round - 1) & 1, abort_flag)) {
                         ok = false;
@@ -225,102 +327,106 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Abort: let the copies in flight land before the CTA exits.
                 mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
-                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
+                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx & (C::kStages - 1)]),
                                       (idx / C::kStages) & 1);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------- MMA issuer
-        constexpr uint32_t idS = idesc_bf16_f32(kBlockM, KN, 0);
-        constexpr uint32_t idO = idesc_bf16_f32(kBlockM, D, 1);
-        const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
-        bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->q_full), 0, abort_flag));
-        tc_fence_after();
-        const int total = 2 * it.E;
-        auto wait_full = [&](int idx) {
-            const int s = idx % C::kStages;
-            bool r = __all_sync(0xffffffffu,
-                                mbar_wait(smem_u32(&bar->kv_full[s]), (idx / C::kStages) & 1,
-                                          abort_flag));
+        } else if (warp == 1) {
+            // --------------------------------------------------------- MMA issuer
+            constexpr uint32_t idS = idesc_bf16_f32(kBlockM, KN, 0);
+            constexpr uint32_t idO = idesc_bf16_f32(kBlockM, D, 1);
+            // Descriptors with an empty address field; an operand's start address
+            // (>> 4) is added to the low word, offsets inside a tile are constants.
+            const uint64_t dK = smem_desc_sw128(0, 16, 1024);
+            const uint64_t dV = smem_desc_sw128(0, C::kKVChunk, 1024);
+            const uint32_t q_addr = smem_u32(sQ) >> 4, kv_addr = smem_u32(sKV) >> 4;
+            bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->q_full), 0, abort_flag));
             tc_fence_after();
-            return r;
-        };
-        auto issue_s = [&](int i, int idx) {
-            const uint32_t a0 = sQa + i * C::kQBytes, b0 = sKVa + (idx % C::kStages) * C::kKVBytes;
+            const int total = 2 * it.E;
+            // TMA completion on the barrier makes the stage visible to the MMA (both async
+            // proxy); no tcgen05 fence is needed after these waits.
+            auto wait_full = [&](int idx) {
+                return __all_sync(0xffffffffu,
+                                  mbar_wait(smem_u32(&bar->kv_full[idx & (C::kStages - 1)]),
+                                            (idx / C::kStages) & 1, abort_flag));
+            };
+            auto issue_s = [&](int i, int idx) {
+                const uint64_t a0 = dK + (q_addr + i * (C::kQBytes >> 4));
+                const uint64_t b0 = dK + (kv_addr + (idx & (C::kStages - 1)) * (C::kKVBytes >> 4));
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off_a = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
-                const uint32_t off_b = (kk >> 2) * C::kKVChunk + (kk & 3) * 32;
-                mma_ss(tmem + i * 128, smem_desc_sw128(a0 + off_a, 16, 1024),
-                       smem_desc_sw128(b0 + off_b, 16, 1024), idS, kk > 0);
-            }
-            mma_commit(smem_u32(&bar->s_full[i]));
-        };
-        auto issue_pv = [&](int i, int idx, bool first) {
-            const uint32_t b0 = sKVa + (idx % C::kStages) * C::kKVBytes;
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + i * 128,
+                           a0 + (uint32_t)(((kk >> 2) * C::kQChunk + (kk & 3) * 32) >> 4),
+                           b0 + (uint32_t)(((kk >> 2) * C::kKVChunk + (kk & 3) * 32) >> 4), idS,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(smem_u32(&bar->s_full[i]));
+            };
+            auto issue_pv = [&](int i, int idx, bool first) {
+                const uint64_t b0 = dV + (kv_addr + (idx & (C::kStages - 1)) * (C::kKVBytes >> 4));
 #pragma unroll
-            for (int kk = 0; kk < KN / 16; ++kk)
-                mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
-                       smem_desc_sw128(b0 + kk * 2048, C::kKVChunk, 1024), idO,
-                       (!first || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&bar->o_done[i]));
-        };
-        auto release = [&](int idx) {
-            if (idx + C::kStages < total) mma_commit(smem_u32(&bar->kv_empty[idx % C::kStages]));
-        };
-        int pv[2] = {0, 0};
-        if (ok && it.E > 0) {
-            const uint32_t e0 = it.entry(0);
-            ok = wait_full(0);
-            if (ok && lane == 0) {
-                if (e0 & kEntV0) issue_s(0, 0);
-                if (e0 & kEntV1) issue_s(1, 0);
-                release(0);
-            }
-            __syncwarp();
-        }
-        for (int n = 0; ok && n < it.E; ++n) {
-            const uint32_t e = it.entry(n);
-            const bool has_next = n + 1 < it.E;
-            const uint32_t en = has_next ? it.entry(n + 1) : 0u;
-            if (!(ok = wait_full(2 * n + 1))) break;
-            if (e & kEntV0) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(smem_u32(&bar->p_full[0]), pv[0] & 1, abort_flag));
-                tc_fence_after();
-                if (!ok) break;
-                if (lane == 0) issue_pv(0, 2 * n + 1, pv[0] == 0);
-                ++pv[0];
-            }
-            if (has_next) {
-                if (!(ok = wait_full(2 * n + 2))) break;
-                if (lane == 0 && (en & kEntV0)) issue_s(0, 2 * n + 2);
-            }
-            if (e & kEntV1) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(smem_u32(&bar->p_full[1]), pv[1] & 1, abort_flag));
-                tc_fence_after();
-                if (!ok) break;
-                if (lane == 0) issue_pv(1, 2 * n + 1, pv[1] == 0);
-                ++pv[1];
-            }
-            if (lane == 0) {
-                if (has_next) {
-                    if (en & kEntV1) issue_s(1, 2 * n + 2);
-                    release(2 * n + 2);
+                for (int kk = 0; kk < KN / 16; ++kk)
+                    mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
+                           b0 + (uint32_t)(kk * (2048 >> 4)), idO, (!first || kk > 0) ? 1u : 0u);
+                mma_commit(smem_u32(&bar->o_done[i]));
+            };
+            auto release = [&](int idx) {
+                if (idx + C::kStages < total)
+                    mma_commit(smem_u32(&bar->kv_empty[idx & (C::kStages - 1)]));
+            };
+            int pv0 = 0, pv1 = 0;
+            uint32_t e = it.E > 0 ? it.entry(0) : 0u;
+            if (ok && it.E > 0) {
+                ok = wait_full(0);
+                if (ok && lane == 0) {
+                    if (e & kEntV0) issue_s(0, 0);
+                    if (e & kEntV1) issue_s(1, 0);
+                    release(0);
                 }
-                release(2 * n + 1);
+                __syncwarp();
             }
-            __syncwarp();
+            for (int n = 0; ok && n < it.E; ++n) {
+                const bool has_next = n + 1 < it.E;
+                const uint32_t en = has_next ? it.entry(n + 1) : 0u;
+                if (!(ok = wait_full(2 * n + 1))) break;
+                if (e & kEntV0) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&bar->p_full[0]), pv0 & 1, abort_flag));
+                    tc_fence_after();
+                    if (!ok) break;
+                    if (lane == 0) issue_pv(0, 2 * n + 1, pv0 == 0);
+                    ++pv0;
+                }
+                if (has_next) {
+                    if (!(ok = wait_full(2 * n + 2))) break;
+                    if (lane == 0 && (en & kEntV0)) issue_s(0, 2 * n + 2);
+                }
+                if (e & kEntV1) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&bar->p_full[1]), pv1 & 1, abort_flag));
+                    tc_fence_after();
+                    if (!ok) break;
+                    if (lane == 0) issue_pv(1, 2 * n + 1, pv1 == 0);
+                    ++pv1;
+                }
+                if (lane == 0) {
+                    if (has_next) {
+                        if (en & kEntV1) issue_s(1, 2 * n + 2);
+                        release(2 * n + 2);
+                    }
+                    release(2 * n + 1);
+                }
+                __syncwarp();
+                e = en;
+            }
+            if (!ok) {
+                // Abort: wait for every MMA issued so far before TMEM is freed.
+                if (lane == 0) mma_commit(smem_u32(&bar->drain));
+                __syncwarp();
+                mbar_wait_bounded(smem_u32(&bar->drain), 0);
+            }
         }
-        if (!ok) {
-            // Abort: wait for every MMA issued so far before TMEM is freed.
-            if (lane == 0) mma_commit(smem_u32(&bar->drain));
-            __syncwarp();
-            mbar_wait_bounded(smem_u32(&bar->drain), 0);
-        }
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------------ softmax warpgroups
+        setmaxnreg_inc<kRegsHigh>();
         const int wg = (warp - 4) >> 2, quad = warp & 3, row = quad * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const uint32_t tS = tmem + lane_base + wg * 128;
@@ -346,14 +452,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const uint32_t vbit = wg ? kEntV1 : kEntV0, fbit = wg ? kEntF1 : kEntF0;
+        const float sl2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
         int visit = 0;
         bool ok = true;
+        uint32_t e_next = it.E > 0 ? it.entry(0) : 0u;
         for (int n = 0; n < it.E; ++n) {
-            const uint32_t e = it.entry(n);
+            const uint32_t e = e_next;
+            if (n + 1 < it.E) e_next = it.entry(n + 1);
             if (!(e & vbit)) continue;
-            const bool full = (e & fbit) != 0;
-            const int kc = (int)(e & kEntChunkMask);
             ok = __all_sync(0xffffffffu,
                             mbar_wait(smem_u32(&bar->s_full[wg]), visit & 1, abort_flag));
             tc_fence_after();
@@ -362,78 +469,100 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < KN / 32; ++j)
                 tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[j * 32]));
+            const bool full = (e & fbit) != 0;
+            uint32_t keep[KN / 32];
+            if (!full)  // mask computed while the TMEM load is in flight
+                keep_mask<KN>(korder, type, band, p.anchor, p.F, p.S, p.nk_rows, fq, sq,
+                              (int)(e & kEntChunkMask) * KN, keep);
             tmem_wait_ld();
-            if (!full) {
-                const int k0 = kc * KN;
-                int fk = 0, sk = 0;
-                pos_to_coord(korder, min(k0, p.nk_rows - 1), p.F, p.S, fk, sk);
+
+            // The two instantiations: full tiles carry no mask arithmetic.
+            auto body = [&](auto masked_tag) {
+                constexpr bool kMasked = decltype(masked_tag)::value;
+                if (kMasked) {
 #pragma unroll
-                for (int c = 0; c < KN; ++c) {
-                    bool keep = (k0 + c) < p.nk_rows;
-                    if (type != MASK_DENSE)
-                        keep = keep && keep_pair(type, band, p.anchor, fq, sq, fk, sk);
-                    if (!keep) r[c] = __float_as_uint(-INFINITY);
-                    step_coord(korder, p.F, p.S, fk, sk);
+                    for (int c = 0; c < KN; ++c)
+                        if (!((keep[c >> 5] >> (c & 31)) & 1u)) r[c] = kNegInfBits;
                 }
-            }
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+                float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < KN; c += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(r[c]));
-                mx1 = fmaxf(mx1, __uint_as_float(r[c + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(r[c + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(r[c + 3]));
-            }
-            const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
-            bool need = false;
-            float m_new;
-            if (m_used == -INFINITY) {
-                m_used = m_new = mt;  // O holds only zero rows so far: nothing to rescale
-            } else if (mt > m_used + kRescaleThreshold) {
-                need = true;
-                m_new = mt;
-            } else {
-                m_new = m_used;
-            }
-            if (__any_sync(0xffffffffu, need)) {
-                // O += P V of the previous visit must be complete before O is touched.
-                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->o_done[wg]),
-                                                       (visit - 1) & 1, abort_flag));
-                tc_fence_after();
-                if (!ok) break;
-                const float fac = need ? fast_exp2(m_used - m_new) : 1.f;
-                l *= fac;
-                m_used = m_new;
+                for (int c = 0; c < KN; c += 8) {
+                    a0 = fmax3(a0, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+                    a1 = fmax3(a1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+                    a2 = fmax3(a2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+                    a3 = fmax3(a3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+                }
+                const float mt = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+                bool need = false;
+                float m_new;
+                if (m_used == -INFINITY) {
+                    m_used = m_new = mt;  // O holds only zero rows so far: nothing to rescale
+                } else if (mt > m_used + kRescaleThreshold) {
+                    need = true;
+                    m_new = mt;
+                } else {
+                    m_new = m_used;
+                }
+                if (__any_sync(0xffffffffu, need)) {
+                    // O += P V of the previous visit must be complete before O is touched.
+                    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->o_done[wg]),
+                                                           (visit - 1) & 1, abort_flag));
+                    tc_fence_after();
+                    if (!ok) return;
+                    const float fac = need ? fast_exp2(m_used - m_new) : 1.f;
+                    l *= fac;
+                    m_used = m_new;
 #pragma unroll 1
-                for (int j = 0; j < D / 32; ++j) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + j * 32, o);
-                    tmem_wait_ld();
+                    for (int j = 0; j < D / 32; ++j) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + j * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
-                    tmem_st32(tO + j * 32, o);
+                        for (int c = 0; c < 32; ++c)
+                            o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
+                        tmem_st32(tO + j * 32, o);
+                    }
+                    tmem_wait_st();
                 }
-                tmem_wait_st();
-            }
-            const float ms = (m_used == -INFINITY) ? 0.f : m_used;
-            float sum0 = 0.f, sum1 = 0.f;
+                const float ms = (m_used == -INFINITY) ? 0.f : m_used;
+                const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ms, -ms);
+                float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < KN / 64; ++j) {
-                uint32_t pk[32];
+                for (int j = 0; j < KN / 32; ++j) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float a = fast_exp2(fmaf(__uint_as_float(r[j * 64 + 2 * c]), p.scale_log2, -ms));
-                    const float b = fast_exp2(fmaf(__uint_as_float(r[j * 64 + 2 * c + 1]), p.scale_log2, -ms));
-                    sum0 += a;
-                    sum1 += b;
-                    pk[c] = pack_bf16x2(a, b);
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const int c = j * 32 + 2 * c2;
+                        const float2 x = ffma2(
+                            make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2, nm2);
+                        float2 ev;
+                        if (!kMasked && SVGA_POLY_EVERY > 0 &&
+                            (c2 % (SVGA_POLY_EVERY > 0 ? SVGA_POLY_EVERY : 1)) ==
+                                (SVGA_POLY_EVERY > 0 ? SVGA_POLY_EVERY - 1 : 0))
+                            ev = exp2_poly2(x);
+                        else
+                            ev = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                        if (c2 & 1)
+                            s1 = fadd2(s1, ev);
+                        else
+                            s0 = fadd2(s0, ev);
+                        pk[c2] = pack_bf16x2_int(ev.x, ev.y);
+                    }
+                    tmem_st16(tS + j * 16, pk);
                 }
-                tmem_st32(tS + j * 32, pk);
-            }
+                l += (s0.x + s0.y) + (s1.x + s1.y);
+            };
+            if (full)
+                body(std::false_type{});
+            else
+                body(std::true_type{});
+            if (!ok) break;
             tmem_wait_st();
-            l += sum0 + sum1;
+            // every lane's P is in TMEM (wait::st + fence); after the warp-level sync one
+            // arrival per warp hands the tile to the MMA issuer
             tc_fence_before();
-            mbar_arrive(smem_u32(&bar->p_full[wg]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar->p_full[wg]));
             ++visit;
         }
         // ----------------------------------------------------------------- epilogue
@@ -457,7 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (row_valid) {
                     if (OUT_F32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + j * 32);
+                        float4 *dst =
+                            reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + j * 32);
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv,
@@ -465,14 +595,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  __uint_as_float(o[4 * c + 2]) * inv,
                                                  __uint_as_float(o[4 * c + 3]) * inv);
                     } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow + j * 32);
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow +
+                                                               j * 32);
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            dst[c] = make_uint4(
-                                pack_bf16x2(__uint_as_float(o[8 * c]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+                            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c]) * inv,
+                                                            __uint_as_float(o[8 * c + 1]) * inv),
+                                                pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv,
+                                                            __uint_as_float(o[8 * c + 3]) * inv),
+                                                pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv,
+                                                            __uint_as_float(o[8 * c + 5]) * inv),
+                                                pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv,
+                                                            __uint_as_float(o[8 * c + 7]) * inv));
                     }
                 }
             }
@@ -532,6 +666,18 @@ template <int D, int KN, bool OUT_F32>
 svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
 {
     using C = Cfg<D, KN>;
+    auto kfn = attn_fwd_kernel<D, KN, OUT_F32>;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kfn) != cudaSuccess) {
+        set_error("cudaFuncGetAttributes failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return SVGA_ERR_CUDA;
+    }
+    if (fa.numRegs < kRegsLaunch) {
+        // the setmaxnreg split assumes the CTA is launched with kRegsLaunch registers/thread
+        set_error("attention kernel built with %d registers/thread, the register split needs %d",
+                  fa.numRegs, kRegsLaunch);
+        return SVGA_ERR_UNSUPPORTED;
+    }
     CUtensorMap tq, tk, tv;
     if (!make_tmap(&tq, a.q, a.heads, a.nq_rows, D, kBlockM) ||
         !make_tmap(&tk, a.k, a.heads, a.nk_rows, D, KN) ||
@@ -539,7 +685,6 @@ svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
         set_error("cuTensorMapEncodeTiled failed (driver entry point or arguments)");
         return SVGA_ERR_CUDA;
     }
-    auto kfn = attn_fwd_kernel<D, KN, OUT_F32>;
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) !=
         cudaSuccess) {
         set_error("cudaFuncSetAttribute(max dynamic shared memory) failed");
@@ -576,6 +721,10 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
         const char *plan = static_cast<const char *>(a.plan);
         kp.head_info = reinterpret_cast<const int4 *>(plan + sizeof(PlanHeader));
         kp.items = kp.head_info + a.heads;
+        // entries start after header + head_info + items, 256-byte aligned
+        const size_t hdr =
+            align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)a.heads + a.n_items), 256);
+        kp.entries = reinterpret_cast<const uint32_t *>(plan + hdr);
     } else {
         kp.head_info = reinterpret_cast<const int4 *>(a.head_info);
         kp.items = nullptr;
@@ -585,12 +734,6 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.o = a.o;
     kp.lse = a.lse;
     kp.status = a.status;
-    if (a.mode == 0) {
-        // entries start after header + head_info + items, 256-byte aligned
-        size_t hdr = sizeof(PlanHeader) + sizeof(int4) * ((size_t)a.heads + a.n_items);
-        hdr = align_up(hdr, 256);
-        kp.entries = reinterpret_cast<const uint32_t *>(static_cast<const char *>(a.plan) + hdr);
-    }
     const int d = a.d, kn = a.kn;
     if (d == 128 && kn == 128)
         return a.out_f32 ? launch_t<128, 128, true>(a, kp, st) : launch_t<128, 128, false>(a, kp, st);

@@ -309,11 +309,67 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
+// Two non-negative finite floats to packed bf16 (lo in the low half) on the integer
+// pipes: add half an ulp of bf16 to the bit pattern and keep the upper 16 bits (round to
+// nearest, ties away from zero), then one byte permute.  Used for the softmax
+// probabilities, where the conversion instruction would compete with the exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi)
+{
+    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
 __device__ __forceinline__ float fast_exp2(float x)
 {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of data.  The
+// compiler builtins keep the operands in register pairs without extra moves.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of x in [-125, 64] on the FMA pipe instead of the MUFU unit.
+// Range reduction: n = round(x) through the 1.5 * 2^23 rounding constant, f = x - n in
+// [-0.5, 0.5]; 2^f from a degree-3 polynomial whose coefficients are this library's own
+// minimax fit (Remez exchange on relative error, max 7.5e-5, far below bf16's 2^-9);
+// 2^n is added to the exponent field with one integer multiply-add.
+__device__ __forceinline__ float2 exp2_poly2(float2 x)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2(x, make_float2(kRound, kRound));
+    const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+    const float2 f = fadd2(x, make_float2(-n.x, -n.y));
+    float2 p = ffma2(make_float2(0.05517167f, 0.05517167f), f, make_float2(0.24261113f, 0.24261113f));
+    p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
+    p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
+    const uint32_t rx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+    const uint32_t ry = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 }  // namespace svga
