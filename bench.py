@@ -161,8 +161,28 @@ def run_svga(args, rank, world, local_rank):
     scale = 1.0 / math.sqrt(d)
     q, k, v = make_qkv(wl)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    prob = svga.ProblemSpec.from_workload(wl)
     stream = torch.cuda.current_stream(dev)
+    classify = None
+    if wl.classify_fraction > 0:
+        # online head classification (routing: outside the timed step, timed on its own)
+        n_rows = max(1, int(math.ceil(wl.tokens * wl.classify_fraction)))
+        prob0 = svga.ProblemSpec.from_workload(wl)
+        ws = torch.empty(svga.svga_classify_size(prob0, n_rows), dtype=torch.uint8, device=dev)
+        types, mse = svga.svga_classify_heads(qd, kd, vd, prob0, wl.cand_spatial,
+                                              wl.cand_temporal, None, n_rows, scale, ws)
+        t0 = time.perf_counter()
+        for _ in range(3):
+            types, mse = svga.svga_classify_heads(qd, kd, vd, prob0, wl.cand_spatial,
+                                                  wl.cand_temporal, None, n_rows, scale, ws)
+        classify_ms = (time.perf_counter() - t0) / 3 * 1e3
+        band = [wl.cand_spatial[h] if types[h] == C.SPATIAL else wl.cand_temporal[h]
+                for h in range(H)]
+        order = [C.ORDER_FRAME_MAJOR if t == C.SPATIAL else C.ORDER_TEMPORAL_MAJOR for t in types]
+        wl = C.Workload(**{**wl.__dict__, "head_type": list(types), "band": band,
+                           "order": order})
+        classify = {"ms": classify_ms, "rows_per_head": n_rows, "types": list(types),
+                    "mse": [[round(a, 9), round(b, 9)] for a, b in mse]}
+    prob = svga.ProblemSpec.from_workload(wl)
 
     # block map: built once (timed on its own)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -328,37 +348,49 @@ def run_svga(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if classify is not None:
+        out["classify"] = classify
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, q, k, v, args.cpu_seconds)
     return out
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample(wl, q, k, v, rows_per_head: int, seed: int):
+def as_f32(q, k, v):
+    """Per-head float32 copies for the oracle (bf16 values, exact), made before timing."""
+    return [tuple(np.ascontiguousarray(x[h].float().numpy()) for x in (q, k, v))
+            for h in range(q.shape[0])]
+
+
+def oracle_sample(wl, qkv32, rows_per_head: int, seed: int):
     """Run the oracle on `rows_per_head` rows of every head; returns (seconds, kept FLOP)."""
     import oracle
     rng = np.random.default_rng(seed)
     N = wl.tokens
     rows = np.sort(rng.choice(N, size=rows_per_head, replace=False)).astype(np.int32)
     t = time.perf_counter()
-    flops = 0.0
     for h in range(wl.heads):
-        oracle.attention_rows(q[h].float().numpy(), k[h].float().numpy(), v[h].float().numpy(),
-                              wl.frames, wl.tokens_per_frame, 1.0 / math.sqrt(wl.head_dim),
-                              wl.head_type[h], wl.band[h], wl.anchor_frame0, rows)
-        flops += sum(4.0 * kept_keys_of_row(wl, h, int(r)) * wl.head_dim for r in rows)
-    return time.perf_counter() - t, flops
+        qh, kh, vh = qkv32[h]
+        oracle.attention_rows(qh, kh, vh, wl.frames, wl.tokens_per_frame,
+                              1.0 / math.sqrt(wl.head_dim), wl.head_type[h], wl.band[h],
+                              wl.anchor_frame0, rows)
+    dt = time.perf_counter() - t
+    flops = sum(4.0 * kept_keys_of_row(wl, h, int(r)) * wl.head_dim
+                for h in range(wl.heads) for r in rows)
+    return dt, flops
 
 
-def calibrate_rows(wl, q, k, v, seconds: float) -> int:
-    dt, _ = oracle_sample(wl, q, k, v, 8, 123)
-    return max(8, min(wl.tokens, int(8 * seconds / max(dt, 1e-3))))
+def calibrate_rows(wl, qkv32, seconds: float) -> int:
+    oracle_sample(wl, qkv32, 4, 321)  # first call pays for thread start-up
+    dt, _ = oracle_sample(wl, qkv32, 16, 123)
+    return max(16, min(wl.tokens, int(16 * seconds / max(dt, 1e-3))))
 
 
 def cpu_baseline(wl, q, k, v, seconds: float):
     import oracle
-    rows = calibrate_rows(wl, q, k, v, seconds)
-    dt, fl = oracle_sample(wl, q, k, v, rows, 7)
+    qkv32 = as_f32(q, k, v)
+    rows = calibrate_rows(wl, qkv32, seconds)
+    dt, fl = oracle_sample(wl, qkv32, rows, 7)
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"{rows} query rows per head x {wl.heads} heads of {wl.name} "
@@ -371,12 +403,13 @@ def run_reference(args, rank, world):
         return None
     wl = C.ALL[args.config]()
     q, k, v = make_qkv(wl)
-    rows = calibrate_rows(wl, q, k, v, args.ref_step_seconds)
+    qkv32 = as_f32(q, k, v)
+    rows = calibrate_rows(wl, qkv32, args.ref_step_seconds)
     for i in range(args.warmup):
-        oracle_sample(wl, q, k, v, rows, 1000 + i)
+        oracle_sample(wl, qkv32, rows, 1000 + i)
     tot_t, tot_f = 0.0, 0.0
     for i in range(args.steps):
-        dt, fl = oracle_sample(wl, q, k, v, rows, i)
+        dt, fl = oracle_sample(wl, qkv32, rows, i)
         tot_t += dt
         tot_f += fl
     value = tot_f / tot_t / 1e12

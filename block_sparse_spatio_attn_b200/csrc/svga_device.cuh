@@ -165,6 +165,20 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier over nthreads threads that also returns the OR of every thread's flag,
+// so that all of them take the same decision after it.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool flag)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.or.pred q, %1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(nthreads), "r"((uint32_t)flag)
+        : "memory");
+    return r != 0;
+}
+
 // ---------------------------------------------------------------- tcgen05 glue
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
 {
