@@ -72,6 +72,21 @@ def kept_flops(wl) -> float:
                      for t, w in zip(wl.head_type, wl.band)))
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (the job is as slow as its slowest rank);
+    identity on a single process."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_value(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """TFLOP/s of the whole job: every rank runs the full workload (weak scaling)."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -251,10 +266,7 @@ def run_svga(args, rank, world, local_rank):
     clocks = sampler.stop(local_rank) if rank == 0 else None
     elapsed = t0.elapsed_time(t1)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_evs)
-    if world > 1:
-        t = torch.tensor([elapsed, attn_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed, attn_ms = float(t[0]), float(t[1])
+    elapsed, attn_ms = max_over_ranks([elapsed, attn_ms], dev)
     ms_per_step = elapsed / args.steps
     if bmap.device_status() != 0:
         raise RuntimeError(f"device status {bmap.device_status()} in the timed region")
@@ -303,10 +315,7 @@ def run_svga(args, rank, world, local_rank):
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, = max_over_ranks([e2e_ms], dev)
 
     peaks, peak_src = read_peaks()
     timed_s = elapsed / 1e3
@@ -319,7 +328,8 @@ def run_svga(args, rank, world, local_rank):
         traffic = None
     total_flops = kflops * world
     out = {
-        "metric": METRIC, "value": total_flops / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": weak_scaling_value(kflops, world, ms_per_step),
+        "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -342,7 +352,7 @@ def run_svga(args, rank, world, local_rank):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} {'sustained' if sustained else 'burst'} bf16",
                      "kernel": "attn_fwd_kernel<128,128>", "flops_per_launch": visited_flops},
-        "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": weak_scaling_value(kflops, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * H * N * d * 2,
                 "d2h_bytes_per_step": H * N * d * 2},
         "gpu_launches": launches_per_step * args.steps,
