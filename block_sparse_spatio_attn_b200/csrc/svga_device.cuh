@@ -114,6 +114,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase completes (or the
+// hint, in ns, runs out), so that waiting warps leave their issue slots to working ones.
+constexpr uint32_t kSuspendHintNs = 1000000u;  // 1 ms
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity of `bar` has completed.  Gives up after
 // kWaitLimitNs or as soon as *abort is set; returns false when it gave up, after
 // raising *abort so that every other role of the CTA stops waiting too.
@@ -124,9 +140,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             *abort = 1;
