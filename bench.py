@@ -172,6 +172,9 @@ def run_svga(args, rank, world, local_rank):
     if args.tile:
         tq, tk = (int(x) for x in args.tile.lower().split("x"))
         wl = wl.with_tile(tq, tk)
+    if args.order:
+        wl = wl.with_orders({"fm": C.ORDER_FRAME_MAJOR, "tm": C.ORDER_TEMPORAL_MAJOR,
+                             "strict": C.ORDER_TEMPORAL_MAJOR_STRICT}[args.order])
     H, N, d = wl.heads, wl.tokens, wl.head_dim
     scale = 1.0 / math.sqrt(d)
     q, k, v = make_qkv(wl)
@@ -326,7 +329,6 @@ def run_svga(args, rank, world, local_rank):
                                                 "attention.cu"))
     if traffic is not None and args.config != "headline":
         traffic = None
-    total_flops = kflops * world
     out = {
         "metric": METRIC, "value": weak_scaling_value(kflops, world, ms_per_step),
         "unit": "TFLOP/s",
@@ -444,7 +446,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svga", choices=["svga", "reference"])
     ap.add_argument("--config", default="headline", choices=sorted(C.ALL))
-    ap.add_argument("--tile", default="")
+    ap.add_argument("--tile", default="", help="block-map tile, e.g. 64x64, 128x256")
+    ap.add_argument("--order", default="", choices=["", "fm", "tm", "strict"],
+                    help="token order of the temporal heads (default: the workload's)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
