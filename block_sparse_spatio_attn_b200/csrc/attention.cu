@@ -76,13 +76,12 @@ struct Cfg {
     static constexpr int kQChunk = kBlockM * 128;               // 64 columns x 128 rows
     static constexpr int kKVBytes = KN * D * 2;                  // one K or V chunk
     static constexpr int kKVChunk = KN * 128;                    // 64 columns x KN rows
-    static constexpr int kStages = (kKVBytes >= 32768) ? 4 : 8;
+    static constexpr int kStages = (kKVBytes >= 32768) ? 5 : 8;
     static constexpr int kSmemData = 2 * kQBytes + kStages * kKVBytes;
     static constexpr int kSmemBar = 1024;
     static constexpr int kSmemAlloc = kSmemData + kSmemBar + 1024;  // + alignment slack
     static constexpr int kSmemLaunch = kSmemAlloc < 120 * 1024 ? 120 * 1024 : kSmemAlloc;
     static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
-    static_assert((kStages & (kStages - 1)) == 0, "stage count is a power of two");
 };
 
 struct Barriers {
@@ -309,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int n = 0; n < it.E && ok; ++n) {
                 const int kc = (int)(it.entry(n) & kEntChunkMask);
                 for (int t = 0; t < 2; ++t) {
-                    const int idx = 2 * n + t, s = idx & (C::kStages - 1), round = idx / C::kStages;
+                    const int idx = 2 * n + t, s = idx % C::kStages, round = idx / C::kStages;
                     if (round > 0 &&
                         !mbar_wait(smem_u32(&bar->kv_empty[s]), (round - 1) & 1, abort_flag)) {
                         ok = false;
@@ -327,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Abort: let the copies in flight land before the CTA exits.
                 mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
-                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx & (C::kStages - 1)]),
+                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
                                       (idx / C::kStages) & 1);
             }
         } else if (warp == 1) {
@@ -346,12 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // proxy); no tcgen05 fence is needed after these waits.
             auto wait_full = [&](int idx) {
                 return __all_sync(0xffffffffu,
-                                  mbar_wait(smem_u32(&bar->kv_full[idx & (C::kStages - 1)]),
+                                  mbar_wait(smem_u32(&bar->kv_full[idx % C::kStages]),
                                             (idx / C::kStages) & 1, abort_flag));
             };
             auto issue_s = [&](int i, int idx) {
                 const uint64_t a0 = dK + (q_addr + i * (C::kQBytes >> 4));
-                const uint64_t b0 = dK + (kv_addr + (idx & (C::kStages - 1)) * (C::kKVBytes >> 4));
+                const uint64_t b0 = dK + (kv_addr + (idx % C::kStages) * (C::kKVBytes >> 4));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + i * 128,
@@ -361,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(smem_u32(&bar->s_full[i]));
             };
             auto issue_pv = [&](int i, int idx, bool first) {
-                const uint64_t b0 = dV + (kv_addr + (idx & (C::kStages - 1)) * (C::kKVBytes >> 4));
+                const uint64_t b0 = dV + (kv_addr + (idx % C::kStages) * (C::kKVBytes >> 4));
 #pragma unroll
                 for (int kk = 0; kk < KN / 16; ++kk)
                     mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
@@ -370,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto release = [&](int idx) {
                 if (idx + C::kStages < total)
-                    mma_commit(smem_u32(&bar->kv_empty[idx & (C::kStages - 1)]));
+                    mma_commit(smem_u32(&bar->kv_empty[idx % C::kStages]));
             };
             int pv0 = 0, pv1 = 0;
             uint32_t e = it.E > 0 ? it.entry(0) : 0u;
