@@ -64,6 +64,11 @@ def _load():
             lib.orc_attention_rows.restype = None
             lib.orc_attention_rows.argtypes = [P, P, P, I, I, I, ctypes.c_double,
                                                I, I, I, P, I, P, P]
+            lib.orc_tile_counts_range.restype = I
+            lib.orc_tile_counts_range.argtypes = [I, I, I, I, I, I, I, I, LL, LL, P]
+            lib.orc_attention_rows_tile_aligned.restype = I
+            lib.orc_attention_rows_tile_aligned.argtypes = [P, P, P, I, I, I, ctypes.c_double,
+                                                            I, I, I, P, LL, LL, P, I, P, P]
             lib.orc_num_threads.restype = I
             lib.orc_num_threads.argtypes = []
             _lib = lib
@@ -137,6 +142,48 @@ def tile_map(type_: int, band: int, anchor: int, order: int, F: int, S: int,
     return {"counts": counts.reshape(nq, nk), "cls": cls.reshape(nq, nk),
             "full_ptr": fptr, "full_idx": fidx[: fptr[-1]].copy(),
             "bnd_ptr": bptr, "bnd_idx": bidx[: bptr[-1]].copy(), "n_q": nq, "n_k": nk}
+
+
+def tile_counts_range(type_: int, band: int, anchor: int, order: int, F: int, S: int,
+                      tq: int, tk: int, i0: int, i1: int) -> np.ndarray:
+    """Kept-element counts [i1 - i0, n_k] of the q-tiles i0 <= i < i1 of one head."""
+    N = F * S
+    nk = -(-N // tk)
+    counts = np.empty((i1 - i0) * nk, np.int64)
+    rc = _load().orc_tile_counts_range(type_, band, anchor, order, F, S, tq, tk, i0, i1,
+                                       _ptr(counts))
+    if rc != 0:
+        raise RuntimeError(f"orc_tile_counts_range failed ({rc})")
+    return counts.reshape(i1 - i0, nk)
+
+
+def q_tiles_of_rows(order: int, F: int, S: int, tq: int, rows) -> np.ndarray:
+    """q-tile index (position in `order` // tq) of each frame-major token in rows."""
+    return np.array([position(order, F, S, int(t) // S, int(t) % S) // tq for t in rows],
+                    np.int64)
+
+
+def attention_rows_tile_aligned(q: np.ndarray, k: np.ndarray, v: np.ndarray, F: int, S: int,
+                                scale: float, order: int, tq: int, tk: int,
+                                counts: np.ndarray, i0: int, rows: np.ndarray):
+    """Tile-aligned (B3) attention of one head: the mask snapped to tiles, i.e. a query
+    keeps every key of each tile (in the head's token order) that holds a kept pair.
+    counts: [n, n_k] kept-element counts of q-tiles i0 .. i0 + n - 1, covering the rows'
+    q-tiles (tile_counts_range / tile_map).  Returns (O [n, d], LSE [n]) in float64."""
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int64)
+    n, d = rows.shape[0], q.shape[1]
+    o = np.empty((n, d), np.float64)
+    lse = np.empty(n, np.float64)
+    rc = _load().orc_attention_rows_tile_aligned(
+        _ptr(q), _ptr(k), _ptr(v), F, S, d, float(scale), order, tq, tk, _ptr(counts), i0,
+        counts.shape[0], _ptr(rows), n, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise RuntimeError(f"orc_attention_rows_tile_aligned failed ({rc})")
+    return o, lse
 
 
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, F: int, S: int,

@@ -102,6 +102,9 @@ void orc_mask(int type, int band, int anchor, int F, int S, uint8_t *mask)
                                                 (int)(k / S), (int)(k % S));
 }
 
+int orc_tile_counts_range(int type, int band, int anchor, int order, int F, int S,
+                          int tq, int tk, long long i0, long long i1, int64_t *counts);
+
 /* Kept-element count of every (q-tile, k-tile) pair of one head whose tokens are
  * laid out in `order`, on the grid padded to whole tiles (padded pairs not kept).
  * counts has n_q * n_k entries, row-major over (q-tile, k-tile). */
@@ -109,15 +112,26 @@ int orc_tile_counts(int type, int band, int anchor, int order, int F, int S,
                     int tq, int tk, int64_t *counts)
 {
     long long N = (long long)F * S;
+    return orc_tile_counts_range(type, band, anchor, order, F, S, tq, tk, 0,
+                                 (N + tq - 1) / tq, counts);
+}
+
+/* The same counts for the q-tiles i0 <= i < i1 only (counts has (i1 - i0) * n_k
+ * entries): what a check of a few query rows of a large problem needs. */
+int orc_tile_counts_range(int type, int band, int anchor, int order, int F, int S,
+                          int tq, int tk, long long i0, long long i1, int64_t *counts)
+{
+    long long N = (long long)F * S;
     long long nq = (N + tq - 1) / tq, nk = (N + tk - 1) / tk;
+    if (i0 < 0 || i1 > nq || i0 > i1) return -3;
     int32_t *fp = (int32_t *)malloc(sizeof(int32_t) * N);
     int32_t *sp = (int32_t *)malloc(sizeof(int32_t) * N);
     if (!fp || !sp) { free(fp); free(sp); return -2; }
     if (orc_order_coords(order, F, S, fp, sp) != 0) { free(fp); free(sp); return -1; }
-    memset(counts, 0, sizeof(int64_t) * nq * nk);
+    memset(counts, 0, sizeof(int64_t) * (i1 - i0) * nk);
 #pragma omp parallel for schedule(dynamic, 1)
-    for (long long i = 0; i < nq; ++i) {
-        int64_t *row = counts + i * nk;
+    for (long long i = i0; i < i1; ++i) {
+        int64_t *row = counts + (i - i0) * nk;
         for (long long q = i * tq; q < (i + 1) * tq && q < N; ++q) {
             int fq = fp[q], sq = sp[q];
             for (long long k = 0; k < N; ++k)
@@ -204,6 +218,76 @@ void orc_attention_rows(const float *q, const float *k, const float *v, int F, i
         free(qd);
         free(acc);
     }
+}
+
+/* Tile-aligned traversal (B3: ainews.tenesys.com, "Co sie zmienilo?" item 4; oossa.com,
+ * opening paragraph: the mask is aligned with the tiles the kernel computes), read as
+ * the mask snapped to tiles: query token t keeps key token u iff the tile
+ * (pos(t) / tq, pos(u) / tk) holds at least one pair the exact mask keeps, pos being
+ * the position in the head's token order.  Then the plain masked softmax over that set.
+ *   counts : kept-element counts of q-tiles i0 .. i0 + n_cnt - 1 (orc_tile_counts_range),
+ *            n_k entries per q-tile; every row's q-tile must lie in that range
+ *   rows, o, lse: as in orc_attention_rows (frame-major token indices).
+ * Returns 0, or -1 when a row's q-tile is outside the counts given. */
+int orc_attention_rows_tile_aligned(const float *q, const float *k, const float *v, int F,
+                                    int S, int d, double scale, int order, int tq, int tk,
+                                    const int64_t *counts, long long i0, long long n_cnt,
+                                    const int32_t *rows, int nrows, double *o, double *lse)
+{
+    long long N = (long long)F * S, nk = (N + tk - 1) / tk;
+    for (int r = 0; r < nrows; ++r) {
+        long long t = rows[r];
+        long long i = orc_position(order, F, S, (int)(t / S), (int)(t % S)) / tq;
+        if (i < i0 || i >= i0 + n_cnt) return -1;
+    }
+    /* k-tile of every frame-major key token */
+    int64_t *ktile = (int64_t *)malloc(sizeof(int64_t) * N);
+    if (!ktile) return -2;
+    for (long long u = 0; u < N; ++u)
+        ktile[u] = orc_position(order, F, S, (int)(u / S), (int)(u % S)) / tk;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * N);
+        double *qd = (double *)malloc(sizeof(double) * d);
+        double *acc = (double *)malloc(sizeof(double) * d);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            long long t = rows[r];
+            long long i = orc_position(order, F, S, (int)(t / S), (int)(t % S)) / tq;
+            const int64_t *crow = counts + (i - i0) * nk;
+            for (int c = 0; c < d; ++c) qd[c] = (double)q[t * d + c];
+            double m = -INFINITY;
+            for (long long u = 0; u < N; ++u) {
+                if (crow[ktile[u]] == 0) {
+                    x[u] = -INFINITY;
+                    continue;
+                }
+                const float *kr = k + u * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qd[c] * (double)kr[c];
+                x[u] = scale * dot;
+                if (x[u] > m) m = x[u];
+            }
+            for (int c = 0; c < d; ++c) acc[c] = 0.0;
+            double l = 0.0;
+            if (m != -INFINITY) {
+                for (long long u = 0; u < N; ++u) {
+                    if (x[u] == -INFINITY) continue;
+                    double p = exp(x[u] - m);
+                    l += p;
+                    const float *vr = v + u * d;
+                    for (int c = 0; c < d; ++c) acc[c] += p * (double)vr[c];
+                }
+            }
+            for (int c = 0; c < d; ++c) o[(long long)r * d + c] = (l > 0.0) ? acc[c] / l : 0.0;
+            lse[r] = (l > 0.0) ? m + log(l) : -INFINITY;
+        }
+        free(x);
+        free(qd);
+        free(acc);
+    }
+    free(ktile);
+    return 0;
 }
 
 int orc_num_threads(void)

@@ -237,6 +237,96 @@ def test_masked_equals_library_sdpa():
         np.testing.assert_allclose(o, _sdpa64(q, k, v, scale, m), rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------- tile-aligned traversal (B3)
+def brute_snapped_mask(t, w, anchor, order, F, S, tq, tk):
+    """Frame-major [N, N] mask of the tile-aligned traversal, built here with numpy: the
+    exact predicate on the coordinates of each position of `order` (the order written
+    as a grid transpose), any-kept per (q-tile, k-tile) through a padded reshape, then
+    every pair of a visited tile kept, mapped back to frame-major tokens."""
+    N = F * S
+    fm = np.arange(N).reshape(F, S)
+    if order == oracle.FRAME_MAJOR:
+        perm = fm.reshape(-1)
+    elif order == oracle.TEMPORAL_ANCHOR_FIRST:
+        perm = np.concatenate([fm[0], fm[1:].T.reshape(-1)])
+    else:
+        perm = fm.T.reshape(-1)
+    f, s = np.divmod(perm, S)
+    c = f if t == oracle.SPATIAL else s
+    keep = np.abs(c[:, None] - c[None, :]) <= w
+    if anchor:
+        keep |= (f == 0)[None, :]
+    nq, nk = -(-N // tq), -(-N // tk)
+    pad = np.zeros((nq * tq, nk * tk), bool)
+    pad[:N, :N] = keep
+    visited = pad.reshape(nq, tq, nk, tk).any(axis=(1, 3))
+    snapped = visited[np.arange(N) // tq][:, np.arange(N) // tk]
+    assert (snapped >= keep).all()      # a superset of the exact kept set
+    out = np.zeros((N, N), bool)
+    out[np.ix_(perm, perm)] = snapped
+    return out
+
+
+@pytest.mark.parametrize("order", [oracle.FRAME_MAJOR, oracle.TEMPORAL_ANCHOR_FIRST,
+                                   oracle.TEMPORAL_STRICT])
+@pytest.mark.parametrize("tq,tk", [(32, 32), (32, 16), (36, 52)])
+def test_tile_aligned_equals_library_sdpa_on_snapped_mask(order, tq, tk):
+    """The tile-aligned oracle equals torch's fp64 SDPA under the snapped mask built
+    independently above (6 frames x 40 tokens; ragged tiles at 32 and 36 x 52).  The
+    snapped mask must differ from both the exact and the all-ones mask here, so that
+    the tile indexing is really exercised."""
+    F, S, d = 6, 40, 16
+    N = F * S
+    g = torch.Generator().manual_seed(21)
+    q, k, v = (torch.randn(N, d, generator=g).to(torch.bfloat16).float().numpy()
+               for _ in range(3))
+    scale = 0.35
+    rows = np.arange(N, dtype=np.int32)
+    nontrivial = 0
+    # without the anchor too: under the strict order every key tile holds frame-0 keys
+    for t, w, a in [(oracle.SPATIAL, 1, 1), (oracle.TEMPORAL, 3, 1), (oracle.TEMPORAL, 3, 0)]:
+        counts = oracle.tile_map(t, w, a, order, F, S, tq, tk)["counts"]
+        o, lse = oracle.attention_rows_tile_aligned(q, k, v, F, S, scale, order, tq, tk,
+                                                    counts, 0, rows)
+        m = brute_snapped_mask(t, w, a, order, F, S, tq, tk)
+        nontrivial += (not m.all()) and (m != oracle.mask(t, w, a, F, S).astype(bool)).any()
+        np.testing.assert_allclose(o, _sdpa64(q, k, v, scale, m), rtol=0, atol=1e-12)
+        x = scale * q.astype(np.float64) @ k.astype(np.float64).T
+        x = np.where(m, x, -np.inf)
+        mx = x.max(1)
+        np.testing.assert_allclose(lse, mx + np.log(np.exp(x - mx[:, None]).sum(1)),
+                                   atol=1e-12)
+    assert nontrivial >= 1
+
+
+def test_tile_aligned_reduces_to_exact_when_frames_fill_tiles():
+    """Frame-major spatial heads whose frames are whole tiles have no boundary tile, so
+    snapping changes nothing: the tile-aligned result is the exact one."""
+    wl = C.tiny()                        # 3 frames of 64 tokens
+    q, k, v = make_qkv(wl)
+    F, S = wl.frames, wl.tokens_per_frame
+    rows = np.arange(F * S, dtype=np.int32)
+    qh, kh, vh = (x[0].float().numpy() for x in (q, k, v))
+    m = oracle.tile_map(oracle.SPATIAL, 1, 1, oracle.FRAME_MAJOR, F, S, 64, 64)
+    assert m["bnd_idx"].size == 0
+    o, lse = oracle.attention_rows_tile_aligned(qh, kh, vh, F, S, 0.125, oracle.FRAME_MAJOR,
+                                                64, 64, m["counts"], 0, rows)
+    oe, le = oracle.attention_rows(qh, kh, vh, F, S, 0.125, oracle.SPATIAL, 1, 1, rows)
+    np.testing.assert_allclose(o, oe, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, le, rtol=0, atol=1e-12)
+
+
+def test_tile_counts_range_is_a_slice_of_the_full_counts():
+    F, S = 3, 40
+    for order in (oracle.FRAME_MAJOR, oracle.TEMPORAL_ANCHOR_FIRST):
+        full = oracle.tile_map(oracle.TEMPORAL, 5, 1, order, F, S, 48, 80)["counts"]
+        np.testing.assert_array_equal(
+            oracle.tile_counts_range(oracle.TEMPORAL, 5, 1, order, F, S, 48, 80, 1, 3),
+            full[1:3])
+    with pytest.raises(RuntimeError):
+        oracle.tile_counts_range(oracle.TEMPORAL, 5, 1, 0, F, S, 48, 80, 2, 9)
+
+
 def test_special_cases():
     F, S, d = 3, 20, 16
     N = F * S
