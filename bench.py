@@ -293,6 +293,25 @@ def run_svga(args, rank, world, local_rank):
                                                               scale, svga.FLAG_NAIVE_B1), reps)
     perm_ms = time_it(lambda: svga.svga_permute_tokens(qd, qp, prob), reps)
     dense_flops = 4.0 * H * N * N * d
+    # tile-aligned traversal (B3, opt-in): every pair of a visited tile is kept
+    b3 = None
+    if wl.tile_q >= 128:
+        # timed alternately with the exact traversal (order swapped each round), so that
+        # both see the same clocks under the power cap
+        b2_t, b3_t = [], []
+        for rnd in range(4):
+            for fl in ((0, svga.FLAG_TILE_ALIGNED) if rnd % 2 == 0 else
+                       (svga.FLAG_TILE_ALIGNED, 0)):
+                t = time_it(lambda: svga.svga_sparse_attention_fwd(
+                    qp, kp, vp, op, None, prob, bmap, scale, fl), max(3, reps // 2))
+                (b3_t if fl else b2_t).append(t)
+        b3_ms, b2_paired_ms = statistics.median(b3_t), statistics.median(b2_t)
+        rq = torch.clamp(N - torch.arange(nq) * wl.tile_q, max=wl.tile_q).double()
+        rk = torch.clamp(N - torch.arange(nk) * wl.tile_k, max=wl.tile_k).double()
+        b3_pairs = float(((cls != 0).double() * (rq[:, None] * rk[None, :])).sum())
+        b3 = {"ms": b3_ms, "exact_b2_ms_alternating": b2_paired_ms,
+              "kept_fraction": b3_pairs / (H * N * N),
+              "tflops_on_kept": 4.0 * d * b3_pairs / (b3_ms * 1e-3) / 1e12}
 
     # -------- end to end through the public API, host buffers ---------------------
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
@@ -349,7 +368,8 @@ def run_svga(args, rank, world, local_rank):
         "boundary_fraction": boundary / (H * nq * nk),
         "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
         "sparse_over_dense": attn_ms / dense_ms, "target_ratio": kept_frac + 0.15,
-        "naive_b1_ms": naive_ms, "permute_ms_per_tensor": perm_ms, "map_build_ms": map_ms,
+        "naive_b1_ms": naive_ms, "tile_aligned_b3": b3,
+        "permute_ms_per_tensor": perm_ms, "map_build_ms": map_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} {'sustained' if sustained else 'burst'} bf16",

@@ -230,9 +230,18 @@ svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *
         set_error("block map plan missing or smaller than svga_block_map_size");
         return SVGA_ERR_INVALID_ARG;
     }
-    if (flags & ~SVGA_FLAG_NAIVE_B1) {
+    if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED)) {
         set_error("unknown flags 0x%x", flags);
         return SVGA_ERR_INVALID_ARG;
+    }
+    if ((flags & SVGA_FLAG_NAIVE_B1) && (flags & SVGA_FLAG_TILE_ALIGNED)) {
+        set_error("SVGA_FLAG_NAIVE_B1 and SVGA_FLAG_TILE_ALIGNED exclude each other");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if ((flags & SVGA_FLAG_TILE_ALIGNED) && problem->tile_q < kBlockM) {
+        // a 128-row query block would hold two query tiles with different key sets
+        set_error("SVGA_FLAG_TILE_ALIGNED needs tile_q >= %d (got %d)", kBlockM, problem->tile_q);
+        return SVGA_ERR_UNSUPPORTED;
     }
     if (!(scale > 0.f) || !(scale < 1e30f)) {
         set_error("scale must be a positive finite number");
@@ -257,6 +266,7 @@ svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *
     a.scale = scale;
     a.mode = 0;
     a.naive = (flags & SVGA_FLAG_NAIVE_B1) ? 1 : 0;
+    a.aligned = (flags & SVGA_FLAG_TILE_ALIGNED) ? 1 : 0;
     a.kn = g.kn;
     a.plan = map->plan;
     a.n_items = g.n_items;

@@ -60,7 +60,7 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "regis
 struct KParams {
     int heads, nq_rows, nk_rows, F, S, anchor;
     float scale_log2;
-    int mode, naive, n_pairs, n_qblk, n_kc;
+    int mode, naive, aligned, n_pairs, n_qblk, n_kc;
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -468,11 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < KN / 32; ++j)
                 tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[j * 32]));
-            const bool full = (e & fbit) != 0;
+            const int kc = (int)(e & kEntChunkMask);
+            // Tile-aligned traversal: a visited chunk keeps every key; only a chunk that
+            // runs past the last token still needs its range mask.
+            const bool full = p.aligned ? (kc + 1) * KN <= p.nk_rows : (e & fbit) != 0;
             uint32_t keep[KN / 32];
             if (!full)  // mask computed while the TMEM load is in flight
-                keep_mask<KN>(korder, type, band, p.anchor, p.F, p.S, p.nk_rows, fq, sq,
-                              (int)(e & kEntChunkMask) * KN, keep);
+                keep_mask<KN>(korder, p.aligned ? MASK_DENSE : type, band, p.anchor, p.F, p.S,
+                              p.nk_rows, fq, sq, kc * KN, keep);
             tmem_wait_ld();
 
             // The two instantiations: full tiles carry no mask arithmetic.
@@ -713,6 +716,7 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.scale_log2 = a.scale * kLog2e;
     kp.mode = a.mode;
     kp.naive = a.naive;
+    kp.aligned = a.aligned;
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;

@@ -69,6 +69,7 @@ struct AttnLaunch {
     float scale;
     int mode;                  // 0 plan, 1 dense (implicit), 2 masked everywhere (implicit)
     int naive;                 // plan mode: visit full tiles through the masked path
+    int aligned;               // plan mode: keep every key of a visited tile (mask snapped to tiles)
     int kn;                    // keys per chunk: 64 or 128
     const void *plan;          // device plan (mode 0)
     const int32_t *head_info;  // device int4 per head (modes 0 and 2)

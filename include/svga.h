@@ -76,7 +76,16 @@ enum {
      * the first sparse kernel of the pages, which masked exactly inside every
      * visited tile (aihirek.info, section "A TPU-kernel kialakitasa dontonek
      * bizonyult"; ainews.tenesys.com, "Co sie zmienilo?" item 1). */
-    SVGA_FLAG_NAIVE_B1 = 1
+    SVGA_FLAG_NAIVE_B1 = 1,
+    /* Tile-aligned traversal (B3): the mask is snapped to the tiles of the block map,
+     * so a query keeps every key of every visited tile, and no visited tile is masked
+     * element by element (ainews.tenesys.com, "Co sie zmienilo?" item 4: the final
+     * "tile-aligned" sparse traversal; oossa.com, opening paragraph: the kernel aligns
+     * the attention mask with the tiles it computes).  The kept set then depends on
+     * order[h] and the tile size and is a superset of the exact one; the result is the
+     * plain masked softmax over that set.  Needs tile_q >= 128 (SVGA_ERR_UNSUPPORTED
+     * otherwise); cannot be combined with SVGA_FLAG_NAIVE_B1 (SVGA_ERR_INVALID_ARG). */
+    SVGA_FLAG_TILE_ALIGNED = 2
 };
 
 /* The problem.  Host struct; the arrays it points to are HOST arrays of `heads`
@@ -201,7 +210,7 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  *   lse        : DEVICE float [heads, tokens] or NULL
  *   map        : built by svga_build_block_map for this same problem
  *   scale      : softmax scale, usually 1/sqrt(head_dim)
- *   flags      : 0 or SVGA_FLAG_NAIVE_B1
+ *   flags      : 0, SVGA_FLAG_NAIVE_B1 or SVGA_FLAG_TILE_ALIGNED
  * bf16 inputs, fp32 accumulation and softmax, P rounded to bf16 for the PV product. */
 SVGA_API svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
                                       float *lse, const svga_problem *problem,

@@ -22,8 +22,9 @@ def problem_of(wl, order=None, tile_q=None, tile_k=None):
 
 
 def run_sparse_path(wl, q, k, v, naive=False, order=None, tile_q=None, tile_k=None,
-                    with_lse=True):
+                    with_lse=True, flags=None):
     """Frame-major Q/K/V on the GPU -> permute -> block-sparse attention -> unpermute.
+    flags overrides `naive` when given.
     Returns (O frame-major bf16 [H,N,d], LSE in each head's order [H,N] or None, map)."""
     from block_sparse_spatio_attn_b200 import svga
     prob = problem_of(wl, order, tile_q, tile_k)
@@ -34,9 +35,10 @@ def run_sparse_path(wl, q, k, v, naive=False, order=None, tile_q=None, tile_k=No
     op = torch.empty_like(q)
     lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) \
         if with_lse else None
+    if flags is None:
+        flags = svga.FLAG_NAIVE_B1 if naive else 0
     svga.svga_sparse_attention_fwd(qp, kp, vp, op, lse, prob, bmap,
-                                   1.0 / math.sqrt(wl.head_dim),
-                                   svga.FLAG_NAIVE_B1 if naive else 0)
+                                   1.0 / math.sqrt(wl.head_dim), flags)
     o = torch.empty_like(q)
     svga.svga_unpermute_tokens(op, o, prob)
     torch.cuda.synchronize()
@@ -62,6 +64,25 @@ def oracle_rows(wl, q, k, v, h, rows, type_=None, band=None):
     return oracle.attention_rows(q[h].float().numpy(), k[h].float().numpy(),
                                  v[h].float().numpy(), F, S, 1.0 / math.sqrt(wl.head_dim),
                                  t, w, wl.anchor_frame0, np.asarray(rows, np.int32))
+
+
+def oracle_rows_tile_aligned(wl, q, k, v, h, rows, order, tq, tk):
+    """Oracle O, LSE of head h under the tile-aligned (snapped) mask, for frame-major
+    rows; the kept-element counts are taken for each group of rows sharing a q-tile."""
+    F, S = wl.frames, wl.tokens_per_frame
+    rows = np.asarray(rows, np.int32)
+    qt = oracle.q_tiles_of_rows(order, F, S, tq, rows)
+    o = np.empty((rows.size, wl.head_dim))
+    lse = np.empty(rows.size)
+    args = [x[h].float().numpy() for x in (q, k, v)]
+    for i in np.unique(qt):
+        sel = np.nonzero(qt == i)[0]
+        counts = oracle.tile_counts_range(wl.head_type[h], wl.band[h], wl.anchor_frame0, order,
+                                          F, S, tq, tk, int(i), int(i) + 1)
+        o[sel], lse[sel] = oracle.attention_rows_tile_aligned(
+            *args, F, S, 1.0 / math.sqrt(wl.head_dim), order, tq, tk, counts, int(i),
+            rows[sel])
+    return o, lse
 
 
 def assert_attn_close(o_gpu: np.ndarray, o_ref: np.ndarray, lse_gpu=None, lse_ref=None,

@@ -20,7 +20,7 @@ if not torch.cuda.is_available():
 
 from block_sparse_spatio_attn_b200 import svga  # noqa: E402
 from tests.helpers import (assert_attn_close, lse_to_frame_major, oracle_rows,  # noqa: E402
-                           run_sparse_path, sample_rows)
+                           oracle_rows_tile_aligned, run_sparse_path, sample_rows)
 
 _cache = {}
 
@@ -166,3 +166,72 @@ def test_repeatable_bitwise():
     o1, l1, _ = run_sparse_path(wl, qd, kd, vd)
     o2, l2, _ = run_sparse_path(wl, qd, kd, vd)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ------------------------------------------------- tile-aligned traversal (B3, opt-in)
+def check_tile_aligned(wl, rows=None, order=None, tile_q=None, tile_k=None):
+    q, k, v, qd, kd, vd = inputs(wl)
+    order = wl.order if order is None else order
+    tq = wl.tile_q if tile_q is None else tile_q
+    tk = wl.tile_k if tile_k is None else tile_k
+    o, lse, _ = run_sparse_path(wl, qd, kd, vd, order=order, tile_q=tq, tile_k=tk,
+                                flags=svga.FLAG_TILE_ALIGNED)
+    o = o.float().cpu().numpy()
+    lse = lse_to_frame_major(lse.cpu().numpy(), wl, order)
+    rows = np.arange(wl.tokens, dtype=np.int32) if rows is None else rows
+    for h in range(wl.heads):
+        ro, rl = oracle_rows_tile_aligned(wl, q, k, v, h, rows, order[h], tq, tk)
+        assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"{wl.name} B3 head {h}")
+
+
+def test_tiny_tile_aligned_all_rows():
+    check_tile_aligned(C.tiny(), tile_q=128, tile_k=64)
+
+
+@pytest.mark.parametrize("tq,tk", [(128, 128), (256, 128), (128, 64), (256, 256)])
+def test_mid_tile_aligned_sampled(tq, tk):
+    wl = C.mid()
+    check_tile_aligned(wl, rows=sample_rows(wl, 300), tile_q=tq, tile_k=tk)
+
+
+def test_mid_tile_aligned_frame_major_temporal():
+    """Temporal heads left frame-major: most visited tiles are boundary tiles there, so
+    snapping keeps many more pairs than the exact mask."""
+    wl = C.mid()
+    check_tile_aligned(wl, rows=sample_rows(wl, 200), order=[C.ORDER_FRAME_MAJOR] * wl.heads)
+
+
+def test_headline_tile_aligned():
+    """Headline size: rows of three q-tiles per head against the oracle (the first, a
+    middle one and the ragged last one)."""
+    wl = C.headline()
+    q, k, v, qd, kd, vd = inputs(wl)
+    F, S = wl.frames, wl.tokens_per_frame
+    o3, l3, _ = run_sparse_path(wl, qd, kd, vd, flags=svga.FLAG_TILE_ALIGNED)
+    n_q = -(-wl.tokens // wl.tile_q)
+    o3n = o3.float().cpu().numpy()
+    for h in range(wl.heads):
+        pos_of_row = np.empty(wl.tokens, np.int64)
+        pos_of_row[oracle.permutation(wl.order[h], F, S)] = np.arange(wl.tokens)
+        qt = pos_of_row // wl.tile_q
+        rows = []
+        for i in (0, n_q // 2, n_q - 1):
+            rr = np.nonzero(qt == i)[0]
+            rows.extend(rr[:: max(1, rr.size // 12)].tolist())
+        rows = np.array(sorted(rows), np.int32)
+        ro, rl = oracle_rows_tile_aligned(wl, q, k, v, h, rows, wl.order[h], wl.tile_q,
+                                          wl.tile_k)
+        lse = lse_to_frame_major(l3[h:h + 1].cpu().numpy(), wl, [wl.order[h]])[0]
+        assert_attn_close(o3n[h, rows], ro, lse[rows], rl, what=f"headline B3 head {h}")
+
+
+def test_tile_aligned_flag_validation():
+    wl = C.tiny()
+    q, k, v, qd, kd, vd = inputs(wl)
+    with pytest.raises(svga.SvgaError) as e:
+        run_sparse_path(wl, qd, kd, vd, tile_q=64, tile_k=128, flags=svga.FLAG_TILE_ALIGNED)
+    assert e.value.status == 4
+    for bad in (svga.FLAG_TILE_ALIGNED | svga.FLAG_NAIVE_B1, 4):
+        with pytest.raises(svga.SvgaError) as e:
+            run_sparse_path(wl, qd, kd, vd, flags=bad)
+        assert e.value.status == 1
