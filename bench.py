@@ -234,6 +234,35 @@ def run_svga(args, rank, world, local_rank):
         svga.svga_unpermute_tokens(op, o, prob)
 
     launches_per_step = 5
+    if args.mode == "parts":
+        # study of one problem split over P GPUs: each part timed alone on this GPU,
+        # which is the whole of what one of P GPUs would run (no exchange between parts)
+        step()
+        torch.cuda.synchronize()
+
+        def med_ms(fn, n=max(3, args.steps)):
+            for _ in range(2):
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n)]
+            for a_, b_ in evs:
+                a_.record(stream)
+                fn()
+                b_.record(stream)
+            torch.cuda.synchronize()
+            return statistics.median(a_.elapsed_time(b_) for a_, b_ in evs)
+
+        single = med_ms(lambda: svga.svga_sparse_attention_fwd(qp, kp, vp, op, None, prob, bmap,
+                                                               scale))
+        part_ms = [med_ms(lambda r=r: svga.svga_sparse_attention_fwd_part(
+            qp, kp, vp, op, None, prob, bmap, scale, 0, r, args.parts))
+            for r in range(args.parts)]
+        if bmap.device_status() != 0:
+            raise RuntimeError(f"device status {bmap.device_status()}")
+        return {"study": "one problem in parts", "workload": wl.name, "parts": args.parts,
+                "single_call_ms": single, "part_ms": part_ms, "max_part_ms": max(part_ms),
+                "projected_speedup": single / max(part_ms),
+                "balance": min(part_ms) / max(part_ms)}
     if args.mode == "attn":
         # profiling aid: the attention kernel alone, warm-up + steps launches, no report
         step()
@@ -472,7 +501,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="full", choices=["full", "attn"],
+    ap.add_argument("--parts", type=int, default=8, help="number of parts for --mode parts")
+    ap.add_argument("--mode", default="full", choices=["full", "attn", "parts"],
                     help="attn: only launch the attention kernel (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -211,11 +211,18 @@ svga_status svga_unpermute_tokens(const void *src, void *dst, const svga_problem
     return permute_common(src, dst, problem, stream, 1);
 }
 
-svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
-                                      float *lse, const svga_problem *problem,
-                                      const svga_block_map *map, float scale, int flags,
-                                      svga_stream_t stream)
+namespace {
+
+svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const svga_problem *problem, const svga_block_map *map,
+                              float scale, int flags, int part, int num_parts,
+                              svga_stream_t stream)
 {
+    if (num_parts < 1 || num_parts > kMaxParts || part < 0 || part >= num_parts) {
+        set_error("part %d of %d: need 1 <= num_parts <= %d and 0 <= part < num_parts", part,
+                  num_parts, kMaxParts);
+        return SVGA_ERR_INVALID_ARG;
+    }
     Geometry g;
     svga_status rc = validate_problem(problem, &g);
     if (rc != SVGA_OK) return rc;
@@ -270,8 +277,29 @@ svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *
     a.kn = g.kn;
     a.plan = map->plan;
     a.n_items = g.n_items;
+    a.part = part;
+    a.num_parts = num_parts;
     a.status = map->status;
     return launch_attention(a, stream);
+}
+
+}  // namespace
+
+svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                                      float *lse, const svga_problem *problem,
+                                      const svga_block_map *map, float scale, int flags,
+                                      svga_stream_t stream)
+{
+    return sparse_fwd_common(q, k, v, o, lse, problem, map, scale, flags, 0, 1, stream);
+}
+
+svga_status svga_sparse_attention_fwd_part(const void *q, const void *k, const void *v, void *o,
+                                           float *lse, const svga_problem *problem,
+                                           const svga_block_map *map, float scale, int flags,
+                                           int part, int num_parts, svga_stream_t stream)
+{
+    return sparse_fwd_common(q, k, v, o, lse, problem, map, scale, flags, part, num_parts,
+                             stream);
 }
 
 svga_status svga_dense_attention_fwd(const void *q, const void *k, const void *v, void *o,

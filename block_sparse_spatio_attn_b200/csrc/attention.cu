@@ -61,6 +61,7 @@ struct KParams {
     int heads, nq_rows, nk_rows, F, S, anchor;
     float scale_log2;
     int mode, naive, aligned, n_pairs, n_qblk, n_kc;
+    int n_items, part, num_parts;  // plan mode: this launch runs the items of one part
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -116,6 +117,15 @@ struct Item {
     }
 };
 
+// Plan items (sorted longest first) are dealt to the parts in snake order: in group g of
+// num_parts consecutive items, part r takes item r when g is even and num_parts-1-r when
+// g is odd, which keeps the parts' total work within one item of each other.
+__device__ __forceinline__ int plan_item_of_block(const KParams &p)
+{
+    const int g = blockIdx.x, r = p.part, n = p.num_parts;
+    return g * n + ((g & 1) ? n - 1 - r : r);
+}
+
 __device__ __forceinline__ Item make_item(const KParams &p, int kn)
 {
     Item it;
@@ -124,7 +134,7 @@ __device__ __forceinline__ Item make_item(const KParams &p, int kn)
     it.n_kc = p.n_kc;
     it.ragged = (p.nk_rows % kn) != 0;
     if (p.mode == 0) {
-        const int4 x = __ldg(p.items + blockIdx.x);
+        const int4 x = __ldg(p.items + plan_item_of_block(p));
         it.h = x.x;
         it.b0 = x.y;
         it.ent = p.entries + x.z;
@@ -264,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (p.mode == 0 && plan_item_of_block(p) >= p.n_items) return;  // the last group ran out
     const Item it = make_item(p, KN);
 
     if (threadIdx.x == 0) {
@@ -692,7 +703,8 @@ svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
         set_error("cudaFuncSetAttribute(max dynamic shared memory) failed");
         return SVGA_ERR_CUDA;
     }
-    if (a.n_items > 0) kfn<<<a.n_items, kThreads, C::kSmemLaunch, st>>>(tq, tk, tv, kp);
+    const int grid = a.mode == 0 ? (a.n_items + kp.num_parts - 1) / kp.num_parts : a.n_items;
+    if (grid > 0) kfn<<<grid, kThreads, C::kSmemLaunch, st>>>(tq, tk, tv, kp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("attention launch failed: %s", cudaGetErrorString(e));
@@ -717,6 +729,9 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.mode = a.mode;
     kp.naive = a.naive;
     kp.aligned = a.aligned;
+    kp.n_items = a.n_items;
+    kp.part = a.part;
+    kp.num_parts = a.num_parts > 0 ? a.num_parts : 1;
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;

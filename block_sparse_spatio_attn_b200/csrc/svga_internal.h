@@ -14,7 +14,8 @@ enum { MASK_SPATIAL = 0, MASK_TEMPORAL = 1, MASK_DENSE = 2 };
 
 constexpr int kMaxHeads = 4096;
 constexpr int kMaxTokens = 1 << 24;
-constexpr int kBlockM = 128;  // query rows per tcgen05 tile (one TMEM lane per row)
+constexpr int kBlockM = 128;
+constexpr int kMaxParts = 4096;  // largest num_parts of a partitioned attention call  // query rows per tcgen05 tile (one TMEM lane per row)
 
 // Execution plan of the attention kernel, stored in svga_block_map::plan.
 //   PlanHeader, then int4 head_info[heads] = {mask type, band, order, 0},
@@ -70,6 +71,7 @@ struct AttnLaunch {
     int mode;                  // 0 plan, 1 dense (implicit), 2 masked everywhere (implicit)
     int naive;                 // plan mode: visit full tiles through the masked path
     int aligned;               // plan mode: keep every key of a visited tile (mask snapped to tiles)
+    int part, num_parts;       // plan mode: run only the items of part `part` (0 of 1: all)
     int kn;                    // keys per chunk: 64 or 128
     const void *plan;          // device plan (mode 0)
     const int32_t *head_info;  // device int4 per head (modes 0 and 2)

@@ -27,7 +27,8 @@ FLAG_TILE_ALIGNED = 2
 
 EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",
             "svga_permute_tokens",
-            "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_dense_attention_fwd",
+            "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_sparse_attention_fwd_part",
+            "svga_dense_attention_fwd",
             "svga_classify_size", "svga_classify_heads", "svga_last_error",
             "svga_status_string", "svga_version"]
 
@@ -80,6 +81,8 @@ def load() -> ctypes.CDLL:
         lib.svga_unpermute_tokens.argtypes = [P, P, PP, P]
         lib.svga_sparse_attention_fwd.argtypes = [P, P, P, P, P, PP, ctypes.POINTER(BlockMapC),
                                                   F, I, P]
+        lib.svga_sparse_attention_fwd_part.argtypes = [P, P, P, P, P, PP,
+                                                      ctypes.POINTER(BlockMapC), F, I, I, I, P]
         lib.svga_dense_attention_fwd.argtypes = [P, P, P, P, P, I, I, I, F, P, P]
         lib.svga_classify_size.argtypes = [PP, I, ctypes.POINTER(SZ)]
         lib.svga_classify_heads.argtypes = [P, P, P, PP, P, P, P, I, F, P, P, P, SZ, P]
@@ -215,6 +218,16 @@ def svga_sparse_attention_fwd(q, k, v, o, lse, problem: ProblemSpec, bmap: Block
     _check(load().svga_sparse_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                             ctypes.byref(problem.c), ctypes.byref(bmap.c),
                                             float(scale), int(flags), _stream(stream)))
+    return o
+
+
+def svga_sparse_attention_fwd_part(q, k, v, o, lse, problem: ProblemSpec, bmap: BlockMap,
+                                   scale: float, flags: int, part: int, num_parts: int,
+                                   stream=None) -> torch.Tensor:
+    _check(load().svga_sparse_attention_fwd_part(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(problem.c),
+        ctypes.byref(bmap.c), float(scale), int(flags), int(part), int(num_parts),
+        _stream(stream)))
     return o
 
 

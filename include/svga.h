@@ -217,6 +217,25 @@ SVGA_API svga_status svga_sparse_attention_fwd(const void *q, const void *k, con
                                       const svga_block_map *map, float scale, int flags,
                                       svga_stream_t stream);
 
+/* One part of svga_sparse_attention_fwd, for running one problem on several GPUs
+ * (or streams) with no exchange between them.  The work items of the block map (a
+ * head and two 128-row query blocks each, longest first) are dealt to num_parts parts
+ * in snake order (group g of num_parts consecutive items: part r takes the r-th item
+ * when g is even, the (num_parts-1-r)-th when g is odd), so that the parts' work
+ * differs by at most about one item.  The call computes and stores the O rows (and
+ * lse entries) of its own items only; the parts of 0 .. num_parts-1 together write
+ * every row exactly once, with results identical bit for bit to the single call.
+ * Heads and query rows are independent in the method (aihirek.info, section
+ * "A Sparse VideoGen a figyelmi fejeket osztalyozza": masks are per head and per
+ * query), so the split needs no communication.  Arguments as for
+ * svga_sparse_attention_fwd, plus
+ *   part, num_parts : 1 <= num_parts <= 4096, 0 <= part < num_parts
+ *                     (SVGA_ERR_INVALID_ARG otherwise). */
+SVGA_API svga_status svga_sparse_attention_fwd_part(const void *q, const void *k, const void *v,
+                                           void *o, float *lse, const svga_problem *problem,
+                                           const svga_block_map *map, float scale, int flags,
+                                           int part, int num_parts, svga_stream_t stream);
+
 /* Dense attention forward (every pair kept): the same-GPU dense baseline, the role
  * dense Splash Attention plays on the pages (aihirek.info, section "A TPU-kernel
  * kialakitasa ..."; oossa.com, "Die Fakten").  Same kernel, every tile unmasked

@@ -235,3 +235,66 @@ def test_tile_aligned_flag_validation():
         with pytest.raises(svga.SvgaError) as e:
             run_sparse_path(wl, qd, kd, vd, flags=bad)
         assert e.value.status == 1
+
+
+# ----------------------------------------------------- one problem split into parts
+def run_parts(wl, num_parts, flags=0):
+    """Every part into its own NaN-filled buffers; returns (single-call O, LSE, per-part
+    O list, per-part LSE list), all in each head's token order."""
+    q, k, v, qd, kd, vd = inputs(wl)
+    prob = svga.ProblemSpec.from_workload(wl)
+    bmap = svga.build_block_map(prob)
+    qp, kp, vp = (torch.empty_like(x) for x in (qd, kd, vd))
+    for s, d in ((qd, qp), (kd, kp), (vd, vp)):
+        svga.svga_permute_tokens(s, d, prob)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    o = torch.empty_like(qd)
+    lse = torch.empty(wl.heads, wl.tokens, dtype=torch.float32, device="cuda")
+    svga.svga_sparse_attention_fwd(qp, kp, vp, o, lse, prob, bmap, scale, flags)
+    ops, lps = [], []
+    for r in range(num_parts):
+        op = torch.full_like(qd, float("nan"))
+        lp = torch.full_like(lse, float("nan"))
+        svga.svga_sparse_attention_fwd_part(qp, kp, vp, op, lp, prob, bmap, scale, flags, r,
+                                            num_parts)
+        ops.append(op)
+        lps.append(lp)
+    torch.cuda.synchronize()
+    assert bmap.device_status() == 0
+    return o, lse, ops, lps
+
+
+@pytest.mark.parametrize("num_parts", [1, 3, 8])
+def test_mid_parts_write_every_row_once_and_match(num_parts):
+    o, lse, ops, lps = run_parts(C.mid(), num_parts)
+    written = torch.stack([~torch.isnan(op.float()).any(dim=-1) for op in ops])  # [P,H,N]
+    assert (written.sum(0) == 1).all()
+    for op, lp, w in zip(ops, lps, written):
+        assert (torch.isnan(op.float()).all(dim=-1) == ~w).all()   # untouched rows stay NaN
+        assert torch.equal(op[w], o[w])
+        assert torch.equal(lp[w], lse[w])
+        assert torch.isnan(lp[~w]).all()
+
+
+def test_headline_eight_parts_match_single_call():
+    o, lse, ops, lps = run_parts(C.headline(), 8, flags=0)
+    comb = torch.zeros_like(o)
+    count = torch.zeros(o.shape[:2], dtype=torch.int32, device=o.device)
+    for op in ops:
+        w = ~torch.isnan(op.float()).any(dim=-1)
+        comb[w] = op[w]
+        count += w.int()
+    assert (count == 1).all()
+    assert torch.equal(comb, o)
+
+
+def test_part_argument_checks():
+    wl = C.tiny()
+    q, k, v, qd, kd, vd = inputs(wl)
+    prob = svga.ProblemSpec.from_workload(wl)
+    bmap = svga.build_block_map(prob)
+    o = torch.empty_like(qd)
+    for part, n in ((1, 1), (-1, 2), (0, 0), (0, 5000)):
+        with pytest.raises(svga.SvgaError) as e:
+            svga.svga_sparse_attention_fwd_part(qd, kd, vd, o, None, prob, bmap, 0.125, 0, part, n)
+        assert e.value.status == 1
