@@ -29,9 +29,12 @@ static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 static bool valid_tile(int t) { return t == 64 || t == 128 || t == 256; }
 
-// Shape checks shared by every call that takes a problem; per-head arrays are checked
-// only when need_heads is set.
-static svga_status validate_shape(const svga_problem *p, Geometry *g, bool need_heads)
+// Shape checks shared by every call that takes a problem.  Per-head arrays: kHeadsSkip
+// does not look at them, kHeadsRequired needs and checks them, kHeadsIfGiven checks them
+// unless all three are NULL (a problem routed by the classifier on the device).
+enum { kHeadsSkip = 0, kHeadsRequired = 1, kHeadsIfGiven = 2 };
+
+static svga_status validate_shape(const svga_problem *p, Geometry *g, int heads_mode)
 {
     if (!p) {
         set_error("problem is NULL");
@@ -65,7 +68,8 @@ static svga_status validate_shape(const svga_problem *p, Geometry *g, bool need_
         set_error("tile %dx%d unsupported (64, 128 or 256)", p->tile_q, p->tile_k);
         return SVGA_ERR_UNSUPPORTED;
     }
-    if (need_heads) {
+    const bool none_given = p->head_type == nullptr && p->band == nullptr && p->order == nullptr;
+    if (heads_mode == kHeadsRequired || (heads_mode == kHeadsIfGiven && !none_given)) {
         if (!p->head_type || !p->band || !p->order) {
             set_error("head_type, band and order must be host arrays of `heads` entries");
             return SVGA_ERR_INVALID_ARG;
@@ -102,7 +106,10 @@ static svga_status validate_shape(const svga_problem *p, Geometry *g, bool need_
     return SVGA_OK;
 }
 
-svga_status validate_problem(const svga_problem *p, Geometry *g) { return validate_shape(p, g, true); }
+svga_status validate_problem(const svga_problem *p, Geometry *g)
+{
+    return validate_shape(p, g, kHeadsRequired);
+}
 
 size_t plan_header_bytes(const Geometry &g)
 {
@@ -144,8 +151,8 @@ svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes, 
                                 int64_t *full_cap, int64_t *bnd_cap, size_t *plan_bytes,
                                 size_t *workspace_bytes)
 {
-    Geometry g;
-    svga_status rc = validate_problem(problem, &g);
+    Geometry g;  // sizes depend on the geometry only, not on the heads' types
+    svga_status rc = validate_shape(problem, &g, kHeadsIfGiven);
     if (rc != SVGA_OK) return rc;
     const int64_t tiles = (int64_t)g.heads * g.n_q * g.n_k;
     if (cls_bytes) *cls_bytes = (size_t)tiles;
@@ -157,12 +164,9 @@ svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes, 
     return SVGA_OK;
 }
 
-svga_status svga_build_block_map(const svga_problem *problem, svga_block_map *map, void *workspace,
-                                 size_t workspace_bytes, svga_stream_t stream)
+static svga_status check_map_buffers(const Geometry &g, const svga_block_map *map,
+                                     const void *workspace, size_t workspace_bytes)
 {
-    Geometry g;
-    svga_status rc = validate_problem(problem, &g);
-    if (rc != SVGA_OK) return rc;
     if (!map || !map->cls || !map->full_ptr || !map->full_idx || !map->bnd_ptr || !map->bnd_idx ||
         !map->plan || !workspace) {
         set_error("block map buffers and workspace must be non-NULL device pointers");
@@ -179,7 +183,49 @@ svga_status svga_build_block_map(const svga_problem *problem, svga_block_map *ma
                   workspace_bytes, block_map_workspace_bytes(g), map->plan_bytes);
         return SVGA_ERR_WORKSPACE;
     }
+    return SVGA_OK;
+}
+
+static svga_status check_bands(int heads, const int32_t *w_spatial, const int32_t *w_temporal)
+{
+    if (!w_spatial || !w_temporal) {
+        set_error("w_spatial and w_temporal must be host arrays of `heads` entries");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    for (int h = 0; h < heads; ++h)
+        if (w_spatial[h] < 0 || w_spatial[h] > 65535 || w_temporal[h] < 0 || w_temporal[h] > 65535) {
+            set_error("head %d: candidate bands must be in 0..65535", h);
+            return SVGA_ERR_INVALID_ARG;
+        }
+    return SVGA_OK;
+}
+
+svga_status svga_build_block_map(const svga_problem *problem, svga_block_map *map, void *workspace,
+                                 size_t workspace_bytes, svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_problem(problem, &g);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_map_buffers(g, map, workspace, workspace_bytes)) != SVGA_OK) return rc;
     return launch_build_block_map(problem, g, map, workspace, workspace_bytes, stream);
+}
+
+svga_status svga_build_block_map_routed(const svga_problem *problem, const int32_t *head_type_dev,
+                                        const int32_t *w_spatial, const int32_t *w_temporal,
+                                        svga_block_map *map, void *workspace,
+                                        size_t workspace_bytes, svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_bands(g.heads, w_spatial, w_temporal)) != SVGA_OK) return rc;
+    if (!head_type_dev || !aligned(head_type_dev, 4)) {
+        set_error("head_type_dev must be a 4-byte aligned device array of `heads` int32");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if ((rc = check_map_buffers(g, map, workspace, workspace_bytes)) != SVGA_OK) return rc;
+    return launch_build_block_map(problem, g, map, workspace, workspace_bytes, stream,
+                                  head_type_dev, w_spatial, w_temporal);
 }
 
 static svga_status permute_common(const void *src, void *dst, const svga_problem *problem,
@@ -197,6 +243,41 @@ static svga_status permute_common(const void *src, void *dst, const svga_problem
         return SVGA_ERR_INVALID_ARG;
     }
     return launch_permute(src, dst, problem, g, inverse, stream);
+}
+
+static svga_status permute_mapped_common(const void *src, void *dst, const svga_problem *problem,
+                                         const svga_block_map *map, svga_stream_t stream,
+                                         int inverse)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if (!map || !map->plan || map->plan_bytes < plan_header_bytes(g)) {
+        set_error("block map plan missing or smaller than svga_block_map_size");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if ((rc = check_tensor(src, "src")) != SVGA_OK || (rc = check_tensor(dst, "dst")) != SVGA_OK)
+        return rc;
+    const size_t bytes = (size_t)g.heads * g.N * g.d * 2;
+    const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
+    if (s < d + bytes && d < s + bytes) {
+        set_error("src and dst overlap");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    return launch_permute(src, dst, problem, g, inverse, stream,
+                          static_cast<const char *>(map->plan) + sizeof(PlanHeader));
+}
+
+svga_status svga_permute_tokens_mapped(const void *src, void *dst, const svga_problem *problem,
+                                       const svga_block_map *map, svga_stream_t stream)
+{
+    return permute_mapped_common(src, dst, problem, map, stream, 0);
+}
+
+svga_status svga_unpermute_tokens_mapped(const void *src, void *dst, const svga_problem *problem,
+                                         const svga_block_map *map, svga_stream_t stream)
+{
+    return permute_mapped_common(src, dst, problem, map, stream, 1);
 }
 
 svga_status svga_permute_tokens(const void *src, void *dst, const svga_problem *problem,
@@ -223,8 +304,8 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
                   num_parts, kMaxParts);
         return SVGA_ERR_INVALID_ARG;
     }
-    Geometry g;
-    svga_status rc = validate_problem(problem, &g);
+    Geometry g;  // per-head type, band and order are read from the plan on the device
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
     if (rc != SVGA_OK) return rc;
     if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
         (rc = check_tensor(v, "v")) != SVGA_OK || (rc = check_tensor(o, "o")) != SVGA_OK)
@@ -354,7 +435,7 @@ svga_status svga_dense_attention_fwd(const void *q, const void *k, const void *v
 svga_status svga_classify_size(const svga_problem *problem, int n_rows, size_t *workspace_bytes)
 {
     Geometry g;
-    svga_status rc = validate_shape(problem, &g, false);
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
     if (rc != SVGA_OK) return rc;
     if (n_rows < 1 || n_rows > g.N) {
         set_error("n_rows %d outside 1..%d", n_rows, g.N);
@@ -364,14 +445,14 @@ svga_status svga_classify_size(const svga_problem *problem, int n_rows, size_t *
     return SVGA_OK;
 }
 
-svga_status svga_classify_heads(const void *q, const void *k, const void *v,
-                                const svga_problem *problem, const int32_t *w_spatial,
-                                const int32_t *w_temporal, const int32_t *rows, int n_rows,
-                                float scale, int32_t *head_type_out, float *mse_out,
-                                void *workspace, size_t workspace_bytes, svga_stream_t stream)
+static svga_status check_classify(const void *q, const void *k, const void *v,
+                                  const svga_problem *problem, const int32_t *w_spatial,
+                                  const int32_t *w_temporal, const int32_t *rows, int n_rows,
+                                  float scale, const int32_t *head_type_out, const void *workspace,
+                                  size_t workspace_bytes)
 {
     Geometry g;
-    svga_status rc = validate_shape(problem, &g, false);
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
     if (rc != SVGA_OK) return rc;
     if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
         (rc = check_tensor(v, "v")) != SVGA_OK)
@@ -380,15 +461,11 @@ svga_status svga_classify_heads(const void *q, const void *k, const void *v,
         set_error("n_rows %d outside 1..%d", n_rows, g.N);
         return SVGA_ERR_SHAPE;
     }
-    if (!w_spatial || !w_temporal || !head_type_out) {
-        set_error("w_spatial, w_temporal and head_type_out must be host arrays");
+    if ((rc = check_bands(g.heads, w_spatial, w_temporal)) != SVGA_OK) return rc;
+    if (!head_type_out || !aligned(head_type_out, 4)) {
+        set_error("head_type_out missing or not 4-byte aligned");
         return SVGA_ERR_INVALID_ARG;
     }
-    for (int h = 0; h < g.heads; ++h)
-        if (w_spatial[h] < 0 || w_spatial[h] > 65535 || w_temporal[h] < 0 || w_temporal[h] > 65535) {
-            set_error("head %d: candidate bands must be in 0..65535", h);
-            return SVGA_ERR_INVALID_ARG;
-        }
     if (rows && !aligned(rows, 4)) {
         set_error("rows is not 4-byte aligned");
         return SVGA_ERR_ALIGNMENT;
@@ -402,8 +479,38 @@ svga_status svga_classify_heads(const void *q, const void *k, const void *v,
         set_error("workspace missing, not 256-byte aligned or smaller than svga_classify_size");
         return SVGA_ERR_WORKSPACE;
     }
+    return SVGA_OK;
+}
+
+svga_status svga_classify_heads(const void *q, const void *k, const void *v,
+                                const svga_problem *problem, const int32_t *w_spatial,
+                                const int32_t *w_temporal, const int32_t *rows, int n_rows,
+                                float scale, int32_t *head_type_out, float *mse_out,
+                                void *workspace, size_t workspace_bytes, svga_stream_t stream)
+{
+    svga_status rc = check_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
+                                    head_type_out, workspace, workspace_bytes);
+    if (rc != SVGA_OK) return rc;
     return run_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
-                        head_type_out, mse_out, workspace, workspace_bytes, stream);
+                        head_type_out, mse_out, nullptr, 0, workspace, workspace_bytes, stream);
+}
+
+svga_status svga_classify_heads_async(const void *q, const void *k, const void *v,
+                                      const svga_problem *problem, const int32_t *w_spatial,
+                                      const int32_t *w_temporal, const int32_t *rows, int n_rows,
+                                      float scale, int32_t *head_type_dev, float *mse_dev,
+                                      int32_t *status_dev, void *workspace,
+                                      size_t workspace_bytes, svga_stream_t stream)
+{
+    svga_status rc = check_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
+                                    head_type_dev, workspace, workspace_bytes);
+    if (rc != SVGA_OK) return rc;
+    if ((mse_dev && !aligned(mse_dev, 4)) || (status_dev && !aligned(status_dev, 4))) {
+        set_error("mse_dev and status_dev must be 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    return run_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
+                        head_type_dev, mse_dev, status_dev, 1, workspace, workspace_bytes, stream);
 }
 
 const char *svga_last_error(void) { return g_last_error; }

@@ -92,6 +92,31 @@ __global__ void write_plan_header_kernel(PlanHeader hdr, HeadParams hp, int4 *he
     }
 }
 
+// The same from head types on the device (the online classifier's output): the band is
+// the candidate of the chosen type, temporal heads read the anchor-first temporal-major
+// order, spatial heads frame-major.  An invalid type is reported in the status word and
+// the head is treated as spatial.
+struct BandPairs {
+    uint32_t packed[kMaxHeads];  // w_spatial | w_temporal << 16
+};
+
+__global__ void write_plan_header_routed_kernel(PlanHeader hdr, BandPairs bp,
+                                                const int32_t *types, int4 *head_info,
+                                                int32_t *status)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) *reinterpret_cast<PlanHeader *>(head_info - 4) = hdr;
+    for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < hdr.heads; h += gridDim.x * blockDim.x) {
+        int t = types[h];
+        if (t != MASK_SPATIAL && t != MASK_TEMPORAL) {
+            if (status) atomicCAS(status, 0, 1);  // SVGA_ERR_INVALID_ARG
+            t = MASK_SPATIAL;
+        }
+        const uint32_t x = bp.packed[h];
+        const int band = t == MASK_SPATIAL ? (int)(x & 0xFFFFu) : (int)(x >> 16);
+        head_info[h] = make_int4(t, band, t == MASK_SPATIAL ? ORDER_FM : ORDER_TM, 0);
+    }
+}
+
 __device__ __forceinline__ int block_sum(int v, int *red)
 {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -308,7 +333,9 @@ size_t block_map_workspace_bytes(const Geometry &g)
 }
 
 svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svga_block_map *map,
-                                   void *ws, size_t ws_bytes, void *stream_)
+                                   void *ws, size_t ws_bytes, void *stream_,
+                                   const int32_t *types_dev, const int32_t *w_spatial,
+                                   const int32_t *w_temporal)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream_);
     const size_t rows = (size_t)g.heads * g.n_q;
@@ -347,11 +374,19 @@ svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svg
     hdr.n_kc = g.n_kc;
     hdr.n_items = g.n_items;
     hdr.entry_cap = entry_cap;
-    HeadParams local;  // 16 KB: travels as kernel parameters
-    for (int h = 0; h < g.heads; ++h)
-        local.packed[h] = (uint32_t)p->head_type[h] | ((uint32_t)p->order[h] << 2) |
-                          ((uint32_t)p->band[h] << 8);
-    write_plan_header_kernel<<<(g.heads + 255) / 256, 256, 0, st>>>(hdr, local, head_info);
+    if (types_dev) {
+        BandPairs bp;  // 16 KB: travels as kernel parameters
+        for (int h = 0; h < g.heads; ++h)
+            bp.packed[h] = (uint32_t)w_spatial[h] | ((uint32_t)w_temporal[h] << 16);
+        write_plan_header_routed_kernel<<<(g.heads + 255) / 256, 256, 0, st>>>(
+            hdr, bp, types_dev, head_info, map->status);
+    } else {
+        HeadParams local;  // 16 KB: travels as kernel parameters
+        for (int h = 0; h < g.heads; ++h)
+            local.packed[h] = (uint32_t)p->head_type[h] | ((uint32_t)p->order[h] << 2) |
+                              ((uint32_t)p->band[h] << 8);
+        write_plan_header_kernel<<<(g.heads + 255) / 256, 256, 0, st>>>(hdr, local, head_info);
+    }
     classify_tiles_kernel<<<dim3(g.n_q, g.heads), 256, 0, st>>>(g, p->anchor_frame0, head_info,
                                                                 map->cls, full_cnt, bnd_cnt);
     scan_kernel<<<1, 1024, 0, st>>>(full_cnt, (int)rows, map->full_ptr, map->full_cap, map->status);

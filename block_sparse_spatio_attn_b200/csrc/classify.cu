@@ -128,8 +128,9 @@ size_t classify_workspace_bytes(const svga_problem *p, int n_rows)
 
 svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
                          const int32_t *w_spatial, const int32_t *w_temporal, const int32_t *rows,
-                         int n_rows, float scale, int32_t *head_type_out, float *mse_out, void *ws,
-                         size_t ws_bytes, void *stream)
+                         int n_rows, float scale, int32_t *head_type_out, float *mse_out,
+                         int32_t *status_out, int device_out, void *ws, size_t ws_bytes,
+                         void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int H = p->heads, d = p->head_dim, S = p->grid_h * p->grid_w, N = p->num_frames * S;
@@ -210,6 +211,19 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     if (e != cudaSuccess) {
         set_error("classifier reduction launch failed: %s", cudaGetErrorString(e));
         return SVGA_ERR_CUDA;
+    }
+    if (device_out) {
+        // results stay on the device: no host round trip, nothing waits
+        if (cudaMemcpyAsync(head_type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToDevice,
+                            st) != cudaSuccess ||
+            (mse_out && cudaMemcpyAsync(mse_out, mse, sizeof(float) * 2 * H,
+                                        cudaMemcpyDeviceToDevice, st) != cudaSuccess) ||
+            (status_out && cudaMemcpyAsync(status_out, status, sizeof(int32_t),
+                                           cudaMemcpyDeviceToDevice, st) != cudaSuccess)) {
+            set_error("classifier result copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+            return SVGA_ERR_CUDA;
+        }
+        return SVGA_OK;
     }
     int32_t dev_status = 0;
     if (cudaMemcpyAsync(head_type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToHost, st) !=

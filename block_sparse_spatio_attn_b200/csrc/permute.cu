@@ -22,10 +22,11 @@ struct OrderParams {
 template <int VPR>  // 16-byte vectors per row (head_dim / 8)
 __global__ void __launch_bounds__(256) permute_kernel(const uint4 *__restrict__ src,
                                                       uint4 *__restrict__ dst, int N, int F, int S,
-                                                      int inverse, OrderParams op)
+                                                      int inverse, OrderParams op,
+                                                      const int4 *__restrict__ head_info)
 {
     const int h = blockIdx.y;
-    const int order = op.order[h];
+    const int order = head_info ? head_info[h].z : op.order[h];
     const size_t head_off = (size_t)h * N * VPR;
     const int total = N * VPR;
     for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
@@ -48,11 +49,12 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4 *__restrict__ 
 }  // namespace
 
 svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
-                           int inverse, void *stream)
+                           int inverse, void *stream, const void *plan_head_info)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     OrderParams op;
-    for (int h = 0; h < g.heads; ++h) op.order[h] = (uint8_t)p->order[h];
+    const int4 *hi = static_cast<const int4 *>(plan_head_info);
+    for (int h = 0; h < g.heads; ++h) op.order[h] = hi ? 0 : (uint8_t)p->order[h];
     const int vpr = g.d / 8;
     const int total = g.N * vpr;
     int blocks = (total + 255) / 256;
@@ -60,10 +62,12 @@ svga_status launch_permute(const void *src, void *dst, const svga_problem *p, co
     dim3 grid(blocks, g.heads);
     if (vpr == 16)
         permute_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
-                                                 static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op);
+                                                 static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op,
+                                                 hi);
     else
         permute_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
-                                                static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op);
+                                                static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op,
+                                                hi);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("permute launch failed: %s", cudaGetErrorString(e));

@@ -52,13 +52,20 @@ int64_t plan_entry_cap(const Geometry &g);
 size_t align_up(size_t x, size_t a);
 
 // block_map.cu
+// Per-head type, band and order come from the problem's host arrays, or, when types_dev
+// is set, from the device (type) and the two candidate band arrays (band by type; order
+// frame-major for spatial, anchor-first temporal-major for temporal heads).
 svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svga_block_map *map,
-                                   void *ws, size_t ws_bytes, void *stream);
+                                   void *ws, size_t ws_bytes, void *stream,
+                                   const int32_t *types_dev = nullptr,
+                                   const int32_t *w_spatial = nullptr,
+                                   const int32_t *w_temporal = nullptr);
 size_t block_map_workspace_bytes(const Geometry &g);
 
 // permute.cu
+// Per-head order from the problem's host array, or from a plan's head info when set.
 svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
-                           int inverse, void *stream);
+                           int inverse, void *stream, const void *plan_head_info = nullptr);
 
 // attention.cu
 struct AttnLaunch {
@@ -87,6 +94,7 @@ size_t classify_workspace_bytes(const svga_problem *p, int n_rows);
 svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
                          const int32_t *w_spatial, const int32_t *w_temporal,
                          const int32_t *rows, int n_rows, float scale, int32_t *head_type_out,
-                         float *mse_out, void *ws, size_t ws_bytes, void *stream);
+                         float *mse_out, int32_t *status_out, int device_out, void *ws,
+                         size_t ws_bytes, void *stream);
 
 }  // namespace svga

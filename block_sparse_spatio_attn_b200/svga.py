@@ -28,6 +28,8 @@ FLAG_TILE_ALIGNED = 2
 EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",
             "svga_permute_tokens",
             "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_sparse_attention_fwd_part",
+            "svga_classify_heads_async", "svga_build_block_map_routed",
+            "svga_permute_tokens_mapped", "svga_unpermute_tokens_mapped",
             "svga_dense_attention_fwd",
             "svga_classify_size", "svga_classify_heads", "svga_last_error",
             "svga_status_string", "svga_version"]
@@ -86,6 +88,11 @@ def load() -> ctypes.CDLL:
         lib.svga_dense_attention_fwd.argtypes = [P, P, P, P, P, I, I, I, F, P, P]
         lib.svga_classify_size.argtypes = [PP, I, ctypes.POINTER(SZ)]
         lib.svga_classify_heads.argtypes = [P, P, P, PP, P, P, P, I, F, P, P, P, SZ, P]
+        lib.svga_classify_heads_async.argtypes = [P, P, P, PP, P, P, P, I, F, P, P, P, P, SZ, P]
+        lib.svga_build_block_map_routed.argtypes = [PP, P, P, P, ctypes.POINTER(BlockMapC), P,
+                                                   SZ, P]
+        lib.svga_permute_tokens_mapped.argtypes = [P, P, PP, ctypes.POINTER(BlockMapC), P]
+        lib.svga_unpermute_tokens_mapped.argtypes = [P, P, PP, ctypes.POINTER(BlockMapC), P]
         lib.svga_last_error.restype = ctypes.c_char_p
         lib.svga_last_error.argtypes = []
         lib.svga_status_string.restype = ctypes.c_char_p
@@ -262,6 +269,49 @@ def svga_classify_heads(q, k, v, problem: ProblemSpec, w_spatial, w_temporal, ro
                                       types, mse, _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
     return list(types), [[mse[2 * h], mse[2 * h + 1]] for h in range(H)]
+
+
+def svga_classify_heads_async(q, k, v, problem: ProblemSpec, w_spatial, w_temporal, rows,
+                              n_rows, scale: float, head_type_dev: torch.Tensor,
+                              mse_dev: Optional[torch.Tensor] = None,
+                              status_dev: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Head types (and deviations, status) written to device tensors; no synchronisation."""
+    H = problem.heads
+    if workspace is None:
+        workspace = torch.empty(svga_classify_size(problem, n_rows), dtype=torch.uint8,
+                                device=q.device)
+    wsp = (ctypes.c_int32 * H)(*w_spatial)
+    wtp = (ctypes.c_int32 * H)(*w_temporal)
+    _check(load().svga_classify_heads_async(
+        _ptr(q), _ptr(k), _ptr(v), ctypes.byref(problem.c), wsp, wtp, _ptr(rows), int(n_rows),
+        float(scale), _ptr(head_type_dev), _ptr(mse_dev), _ptr(status_dev), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+
+
+def svga_build_block_map_routed(problem: ProblemSpec, head_type_dev: torch.Tensor, w_spatial,
+                                w_temporal, bmap: BlockMap, stream=None) -> BlockMap:
+    H = problem.heads
+    wsp = (ctypes.c_int32 * H)(*w_spatial)
+    wtp = (ctypes.c_int32 * H)(*w_temporal)
+    _check(load().svga_build_block_map_routed(ctypes.byref(problem.c), _ptr(head_type_dev), wsp,
+                                              wtp, ctypes.byref(bmap.c), _ptr(bmap.workspace),
+                                              bmap.workspace.numel(), _stream(stream)))
+    return bmap
+
+
+def svga_permute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
+                               bmap: BlockMap, stream=None) -> torch.Tensor:
+    _check(load().svga_permute_tokens_mapped(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
+                                             ctypes.byref(bmap.c), _stream(stream)))
+    return dst
+
+
+def svga_unpermute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
+                                 bmap: BlockMap, stream=None) -> torch.Tensor:
+    _check(load().svga_unpermute_tokens_mapped(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
+                                               ctypes.byref(bmap.c), _stream(stream)))
+    return dst
 
 
 def version() -> int:

@@ -272,6 +272,52 @@ SVGA_API svga_status svga_classify_heads(const void *q, const void *k, const voi
                                 float scale, int32_t *head_type_out, float *mse_out, void *workspace,
                                 size_t workspace_bytes, svga_stream_t stream);
 
+/* ---- Routed pipeline: the classifier's decision stays on the device -------------
+ * The pages profile the heads online and then run the chosen sparse mask (aihirek.info,
+ * section "A Sparse VideoGen a figyelmi fejeket osztalyozza").  The four calls below
+ * run classification -> block map -> permutation -> attention -> inverse permutation
+ * on one stream without returning to the host in between, so a whole attention layer
+ * can be replayed from one CUDA graph.  Per head: type from the classifier, band =
+ * w_spatial[h] or w_temporal[h] by that type, order = frame-major for spatial heads and
+ * anchor-first temporal-major for temporal heads.  The problem's head_type, band and
+ * order arrays are not read by these calls (they may be NULL); svga_block_map_size and
+ * svga_sparse_attention_fwd(_part) do not read them either. */
+
+/* svga_classify_heads without the host round trip: nothing synchronises.
+ *   head_type_dev : DEVICE int32 [heads], written on `stream`
+ *   mse_dev       : DEVICE float [heads][2] or NULL
+ *   status_dev    : DEVICE int32 or NULL: 0, or the svga_status of a failure found
+ *                   on the device (e.g. a row index outside 0..N-1)
+ * Other arguments and their checks as for svga_classify_heads. */
+SVGA_API svga_status svga_classify_heads_async(const void *q, const void *k, const void *v,
+                                      const svga_problem *problem, const int32_t *w_spatial,
+                                      const int32_t *w_temporal, const int32_t *rows,
+                                      int n_rows, float scale, int32_t *head_type_dev,
+                                      float *mse_dev, int32_t *status_dev, void *workspace,
+                                      size_t workspace_bytes, svga_stream_t stream);
+
+/* svga_build_block_map with the head types read on the device from head_type_dev
+ * (DEVICE int32 [heads], e.g. svga_classify_heads_async's output) and the bands and
+ * orders derived from them as described above.  w_spatial, w_temporal: HOST int32
+ * [heads], 0 .. 65535.  A type other than 0 / 1 on the device sets map->status to
+ * SVGA_ERR_INVALID_ARG (the head is then built as spatial).  The plan records every
+ * head's type, band and order for the calls below.  Same buffers as
+ * svga_build_block_map. */
+SVGA_API svga_status svga_build_block_map_routed(const svga_problem *problem,
+                                        const int32_t *head_type_dev, const int32_t *w_spatial,
+                                        const int32_t *w_temporal, svga_block_map *map,
+                                        void *workspace, size_t workspace_bytes,
+                                        svga_stream_t stream);
+
+/* svga_permute_tokens / svga_unpermute_tokens with each head's order read from the
+ * plan of `map` on the device instead of problem->order. */
+SVGA_API svga_status svga_permute_tokens_mapped(const void *src, void *dst,
+                                       const svga_problem *problem, const svga_block_map *map,
+                                       svga_stream_t stream);
+SVGA_API svga_status svga_unpermute_tokens_mapped(const void *src, void *dst,
+                                         const svga_problem *problem,
+                                         const svga_block_map *map, svga_stream_t stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 SVGA_API const char *svga_last_error(void);
 
