@@ -343,29 +343,58 @@ def run_svga(args, rank, world, local_rank):
               "tflops_on_kept": 4.0 * d * b3_pairs / (b3_ms * 1e-3) / 1e12}
 
     # -------- end to end through the public API, host buffers ---------------------
+    # Pipelined as a serving loop would run it: step i's inputs are copied in on one
+    # stream while step i-1 computes on another, and outputs go out on a third; two sets
+    # of device buffers alternate.  Every step's 774 MB still cross PCIe inside the
+    # timed region.
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     oh = torch.empty_like(q).pin_memory()
+    sets = [(qd, kd, vd, qp, kp, vp, op, o), tuple(torch.empty_like(qd) for _ in range(8))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_done, comp_done, out_done = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(3))
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
+    def layer(bs):
+        bq, bk, bv, bqp, bkp, bvp, bop, bo = bs
+        svga.svga_permute_tokens(bq, bqp, prob)
+        svga.svga_permute_tokens(bk, bkp, prob)
+        svga.svga_permute_tokens(bv, bvp, prob)
+        svga.svga_sparse_attention_fwd(bqp, bkp, bvp, bop, None, prob, bmap, scale)
+        svga.svga_unpermute_tokens(bop, bo, prob)
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_run(n, t0=None, t1=None):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[b])     # set b's inputs are free again
+                if i == 0 and t0 is not None:
+                    t0.record(s_in)
+                for dst, src in zip(sets[b][:3], (qh, kh, vh)):
+                    dst.copy_(src, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            if i >= 2:
+                stream.wait_event(out_done[b])        # set b's output has been read out
+            layer(sets[b])
+            comp_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                oh.copy_(sets[b][7], non_blocking=True)
+                out_done[b].record(s_out)
+        if t1 is not None:
+            t1.record(s_out)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(3, min(args.steps, 10))
-    a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    b.record(stream)
+    e2e_steps = max(4, min(args.steps, 12))
+    e2e_run(e2e_steps, a, b)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
+    if bmap.device_status() != 0:
+        raise RuntimeError(f"device status {bmap.device_status()} in the e2e loop")
     e2e_ms, = max_over_ranks([e2e_ms], dev)
 
     peaks, peak_src = read_peaks()
@@ -405,7 +434,9 @@ def run_svga(args, rank, world, local_rank):
                      "kernel": "attn_fwd_kernel<128,128>", "flops_per_launch": visited_flops},
         "e2e": {"value": weak_scaling_value(kflops, world, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * H * N * d * 2,
-                "d2h_bytes_per_step": H * N * d * 2},
+                "d2h_bytes_per_step": H * N * d * 2,
+                "pipeline": "copy-in, compute and copy-out of successive steps overlap on "
+                            "three streams, two device buffer sets"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
