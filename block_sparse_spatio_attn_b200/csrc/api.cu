@@ -318,7 +318,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
         set_error("block map plan missing or smaller than svga_block_map_size");
         return SVGA_ERR_INVALID_ARG;
     }
-    if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED)) {
+    if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED | SVGA_FLAG_TEST_STALL)) {
         set_error("unknown flags 0x%x", flags);
         return SVGA_ERR_INVALID_ARG;
     }
@@ -355,6 +355,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     a.mode = 0;
     a.naive = (flags & SVGA_FLAG_NAIVE_B1) ? 1 : 0;
     a.aligned = (flags & SVGA_FLAG_TILE_ALIGNED) ? 1 : 0;
+    a.test_stall = (flags & SVGA_FLAG_TEST_STALL) ? 1 : 0;
     a.kn = g.kn;
     a.plan = map->plan;
     a.n_items = g.n_items;

@@ -62,6 +62,7 @@ struct KParams {
     float scale_log2;
     int mode, naive, aligned, n_pairs, n_qblk, n_kc;
     int n_items, part, num_parts;  // plan mode: this launch runs the items of one part
+    int test_stall;                // test hook: the first K chunk is never loaded
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -325,6 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (p.test_stall && idx == 0) {  // nothing ever completes this stage
+                        issued = idx + 1;
+                        continue;
+                    }
                     const uint32_t fb = smem_u32(&bar->kv_full[s]);
                     mbar_arrive_expect_tx(fb, C::kKVBytes);
                     for (int c = 0; c < D / 64; ++c)
@@ -337,8 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Abort: let the copies in flight land before the CTA exits.
                 mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
-                    mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
-                                      (idx / C::kStages) & 1);
+                    if (!(p.test_stall && idx == 0))
+                        mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
+                                          (idx / C::kStages) & 1);
             }
         } else if (warp == 1) {
             // --------------------------------------------------------- MMA issuer
@@ -732,6 +738,7 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.n_items = a.n_items;
     kp.part = a.part;
     kp.num_parts = a.num_parts > 0 ? a.num_parts : 1;
+    kp.test_stall = a.test_stall;
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;

@@ -85,7 +85,12 @@ enum {
      * order[h] and the tile size and is a superset of the exact one; the result is the
      * plain masked softmax over that set.  Needs tile_q >= 128 (SVGA_ERR_UNSUPPORTED
      * otherwise); cannot be combined with SVGA_FLAG_NAIVE_B1 (SVGA_ERR_INVALID_ARG). */
-    SVGA_FLAG_TILE_ALIGNED = 2
+    SVGA_FLAG_TILE_ALIGNED = 2,
+    /* Test hook for the failure path: the first K chunk of every CTA is never loaded,
+     * so the kernel's bounded waits run out (about one second per CTA wave), every role
+     * stops, copies in flight are drained, TMEM is released and map->status reads
+     * SVGA_ERR_TIMEOUT.  O is left unwritten.  The CUDA context stays usable. */
+    SVGA_FLAG_TEST_STALL = 1 << 16
 };
 
 /* The problem.  Host struct; the arrays it points to are HOST arrays of `heads`
