@@ -18,14 +18,16 @@
 //     warpgroups work on different tiles while the tensor core runs the other's MMAs;
 //     operand descriptors are built once and advanced by constant offsets;
 //   * warps 4-7 and 8-11 hold one query row per thread (TMEM lane = row): they read S,
-//     run the online softmax in the exp2 domain with packed fp32x2 arithmetic (part of
-//     the exponentials on the FMA pipe by polynomial, the rest on the MUFU unit), write
-//     P back into TMEM over S, and rescale O in TMEM only when the running maximum grows
-//     by more than 2^8 (P stays <= 256 otherwise);
+//     run the online softmax in the exp2 domain with packed fp32x2 arithmetic and the
+//     MUFU exponential, write P back into TMEM over S as bf16, and rescale O in TMEM
+//     only when the running maximum grows by more than 2^8 (P stays <= 256 otherwise);
 //   * boundary tiles build a 128-bit keep mask per row from the runs of the key chunk
 //     (at most a few intervals per run), then mask with one select per element;
 //   * the producer/MMA warpgroup gives registers to the softmax warpgroups (setmaxnreg);
-//   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated).
+//   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated);
+//   * a launch may run one part of the plan's items (snake order), so one problem can
+//     be split over several GPUs; the tile-aligned traversal (B3) treats every visited
+//     chunk as full.
 //
 // Every mbarrier wait gives up after about a second: the CTA raises a shared abort
 // flag, drains its MMAs and copies, frees TMEM, writes SVGA_ERR_TIMEOUT to the
@@ -40,9 +42,6 @@
 #include "svga_device.cuh"
 #include "svga_internal.h"
 
-#ifndef SVGA_POLY_EVERY
-#define SVGA_POLY_EVERY 0  // one pair of exponentials in this many on the FMA pipe (0: none)
-#endif
 
 namespace svga {
 namespace {
@@ -554,13 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int c = j * 32 + 2 * c2;
                         const float2 x = ffma2(
                             make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2, nm2);
-                        float2 ev;
-                        if (!kMasked && SVGA_POLY_EVERY > 0 &&
-                            (c2 % (SVGA_POLY_EVERY > 0 ? SVGA_POLY_EVERY : 1)) ==
-                                (SVGA_POLY_EVERY > 0 ? SVGA_POLY_EVERY - 1 : 0))
-                            ev = exp2_poly2(x);
-                        else
-                            ev = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                        const float2 ev = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                         if (c2 & 1)
                             s1 = fadd2(s1, ev);
                         else

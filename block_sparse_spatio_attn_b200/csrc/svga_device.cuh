@@ -1,14 +1,11 @@
 // svga_device.cuh -- device helpers of the svga CUDA library (sm_100a only).
 //
-//  * token coordinates: position in a token order -> (frame f, in-frame index s)
-//  * the keep predicate of spatial / temporal heads with the frame-0 anchor
+//  * token coordinates: position in a token order <-> (frame f, in-frame index s), for
+//    the frame-major and temporal-major orders the pages use ("Accelerating
+//    Spatio-Temporal Attention for Video Diffusion on TPUs", ainews.tenesys.com,
+//    "Co sie zmienilo?" item 5)
 //  * thin inline-PTX wrappers: mbarrier, TMA tensor loads, tcgen05 (TMEM alloc,
-//    MMA, commit, ld/st, fences), named barriers, global timer.
-//
-// The masks follow "Accelerating Spatio-Temporal Attention for Video Diffusion on
-// TPUs" (aihirek.info summary, section "A Sparse VideoGen a figyelmi fejeket
-// osztalyozza"): spatial heads keep nearby frames, temporal heads keep nearby
-// in-frame positions, both keep frame 0.
+//    MMA, commit, ld/st, fences), global timer, packed fp32x2 arithmetic.
 #pragma once
 #include <cstdint>
 
@@ -48,17 +45,6 @@ __host__ __device__ __forceinline__ int coord_to_pos(int order, int f, int s, in
     return f == 0 ? s : S + s * (F - 1) + (f - 1);
 }
 
-// Keep predicate M(q, k) on original coordinates.
-__host__ __device__ __forceinline__ bool keep_pair(int type, int band, int anchor, int fq,
-                                                   int sq, int fk, int sk)
-{
-    if (type == MASK_DENSE) return true;
-    if (anchor && fk == 0) return true;
-    int d = (type == MASK_SPATIAL) ? (fq - fk) : (sq - sk);
-    d = d < 0 ? -d : d;
-    return d <= band;
-}
-
 // ------------------------------------------------------------------- PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -80,11 +66,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 __device__ __forceinline__ void fence_barrier_init()
 {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar)
@@ -172,25 +153,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
 __device__ __forceinline__ void prefetch_tmap(const void *tmap)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Named barrier over nthreads threads that also returns the OR of every thread's flag,
-// so that all of them take the same decision after it.
-__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool flag)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\t"
-        "bar.red.or.pred q, %1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(id), "r"(nthreads), "r"((uint32_t)flag)
-        : "memory");
-    return r != 0;
 }
 
 // ---------------------------------------------------------------- tcgen05 glue
@@ -365,27 +327,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// 2^x for a pair of x in [-125, 64] on the FMA pipe instead of the MUFU unit.
-// Range reduction: n = round(x) through the 1.5 * 2^23 rounding constant, f = x - n in
-// [-0.5, 0.5]; 2^f from a degree-3 polynomial whose coefficients are this library's own
-// minimax fit (Remez exchange on relative error, max 7.5e-5, far below bf16's 2^-9);
-// 2^n is added to the exponent field with one integer multiply-add.
-__device__ __forceinline__ float2 exp2_poly2(float2 x)
-{
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 t = fadd2(x, make_float2(kRound, kRound));
-    const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-    const float2 f = fadd2(x, make_float2(-n.x, -n.y));
-    float2 p = ffma2(make_float2(0.05517167f, 0.05517167f), f, make_float2(0.24261113f, 0.24261113f));
-    p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
-    p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
-    const uint32_t rx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-    const uint32_t ry = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 template <uint32_t N>
