@@ -26,36 +26,48 @@ struct Rect {
 };
 
 // Positions [u0, u1) of a grid with period P (major = u / P, minor = u % P) as at
-// most three rectangles.  major_is_f: frames follow the major index; otherwise the
-// in-frame index does and frames follow the minor index plus foff.
-__host__ __device__ __forceinline__ int run_rects(int u0, int u1, int P, bool major_is_f, int foff,
-                                         Rect *r)
+// most three rectangles: the first partial major row (h), the whole rows between (m)
+// and the last partial row (t).  major_is_f: frames follow the major index; otherwise
+// the in-frame index does and frames follow the minor index plus foff.  Returns the
+// valid ones as bits (1 = h, 2 = m, 4 = t).  Fixed slots, not a count, so that the
+// rectangles stay in registers.
+__host__ __device__ __forceinline__ uint32_t run_rects(int u0, int u1, int P, bool major_is_f,
+                                                      int foff, Rect &h, Rect &m, Rect &t)
 {
     const int M0 = u0 / P, m0 = u0 - M0 * P;
     const int M1 = (u1 - 1) / P, m1 = (u1 - 1) - M1 * P;
     auto emit = [&](int Ma, int Mb, int ma, int mb) {
         return major_is_f ? Rect{Ma, Mb, ma, mb} : Rect{ma + foff, mb + foff, Ma, Mb};
     };
-    int n = 0;
     if (M0 == M1) {
-        r[n++] = emit(M0, M0, m0, m1);
-        return n;
+        h = emit(M0, M0, m0, m1);
+        return 1u;
     }
-    r[n++] = emit(M0, M0, m0, P - 1);
-    if (M1 > M0 + 1) r[n++] = emit(M0 + 1, M1 - 1, 0, P - 1);
-    r[n++] = emit(M1, M1, 0, m1);
-    return n;
+    h = emit(M0, M0, m0, P - 1);
+    t = emit(M1, M1, 0, m1);
+    if (M1 > M0 + 1) {
+        m = emit(M0 + 1, M1 - 1, 0, P - 1);
+        return 7u;
+    }
+    return 5u;
 }
 
-// Tokens at positions [a, b) of `order` (0 <= a < b <= N) as at most 4 rectangles.
-__host__ __device__ __forceinline__ int tile_rects(int order, int a, int b, int F, int S, Rect *r)
+// Tokens at positions [a, b) of `order` (0 <= a < b <= N) as at most 4 rectangles in
+// fixed slots: r[0] the frame-0 part of the anchor-first order, r[1..3] the run's
+// head, middle and tail.  Returns the valid slots as bits.
+__host__ __device__ __forceinline__ uint32_t tile_rects(int order, int a, int b, int F, int S,
+                                                       Rect (&r)[4])
 {
-    if (order == ORDER_FM) return run_rects(a, b, S, true, 0, r);
-    if (order == ORDER_TM_STRICT) return run_rects(a, b, F, false, 0, r);
-    int n = 0;  // anchor-first: frame 0 at positions [0, S), then s-major over f = 1..F-1
-    if (a < S) r[n++] = Rect{0, 0, a, (b < S ? b : S) - 1};
-    if (b > S) n += run_rects((a > S ? a : S) - S, b - S, F - 1, false, 1, r + n);
-    return n;
+    if (order == ORDER_FM) return run_rects(a, b, S, true, 0, r[1], r[2], r[3]) << 1;
+    if (order == ORDER_TM_STRICT) return run_rects(a, b, F, false, 0, r[1], r[2], r[3]) << 1;
+    uint32_t mask = 0;  // anchor-first: frame 0 at positions [0, S), then s-major over f >= 1
+    if (a < S) {
+        r[0] = Rect{0, 0, a, (b < S ? b : S) - 1};
+        mask = 1u;
+    }
+    if (b > S)
+        mask |= run_rects((a > S ? a : S) - S, b - S, F - 1, false, 1, r[1], r[2], r[3]) << 1;
+    return mask;
 }
 
 // Does the rectangle pair keep all / any of its (q, k) pairs?
@@ -141,22 +153,25 @@ __global__ void __launch_bounds__(256) classify_tiles_kernel(Geometry g, int anc
     const int qa = i * g.tile_q, qb = min(g.N, qa + g.tile_q);
     const bool qpad = qa + g.tile_q > g.N;
     Rect qr[4];
-    const int nqr = tile_rects(order, qa, qb, g.F, g.S, qr);
+    const uint32_t qm = tile_rects(order, qa, qb, g.F, g.S, qr);
     int nf = 0, nb = 0;
     uint8_t *row = cls + ((size_t)h * g.n_q + i) * g.n_k;
     for (int j = threadIdx.x; j < g.n_k; j += blockDim.x) {
         const int ka = j * g.tile_k, kb = min(g.N, ka + g.tile_k);
         const bool kpad = ka + g.tile_k > g.N;
         Rect kr[4];
-        const int nkr = tile_rects(order, ka, kb, g.F, g.S, kr);
+        const uint32_t km = tile_rects(order, ka, kb, g.F, g.S, kr);
         bool full = !qpad && !kpad, any = false;
-        for (int a = 0; a < nqr; ++a)
-            for (int b = 0; b < nkr; ++b) {
-                bool all_, any_;
-                rect_pair(type, band, anchor, qr[a], kr[b], all_, any_);
-                full = full && all_;
-                any = any || any_;
-            }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (((qm >> a) & 1u) && ((km >> b) & 1u)) {
+                    bool all_, any_;
+                    rect_pair(type, band, anchor, qr[a], kr[b], all_, any_);
+                    full = full && all_;
+                    any = any || any_;
+                }
         const uint8_t c = any ? (full ? 1 : 2) : 0;
         row[j] = c;
         nf += c == 1;
@@ -397,7 +412,8 @@ svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svg
     plan_count_kernel<<<g.n_items, 256, 0, st>>>(g, map->cls, item_cnt);
     scan_kernel<<<1, 1024, 0, st>>>(item_cnt, g.n_items, item_off, entry_cap, map->status);
     plan_write_kernel<<<g.n_items, 256, 0, st>>>(g, map->cls, item_off, entries, entry_cap);
-    plan_sort_kernel<<<(g.n_items + 255) / 256, 256, 0, st>>>(g, item_cnt, item_off, items);
+    // 64-thread blocks: the rank count is O(n) per item, so spread items over many SMs
+    plan_sort_kernel<<<(g.n_items + 63) / 64, 64, 0, st>>>(g, item_cnt, item_off, items);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("block map launch failed: %s", cudaGetErrorString(e));
