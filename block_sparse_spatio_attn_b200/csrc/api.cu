@@ -111,6 +111,11 @@ svga_status validate_problem(const svga_problem *p, Geometry *g)
     return validate_shape(p, g, kHeadsRequired);
 }
 
+svga_status validate_geometry(const svga_problem *p, Geometry *g)
+{
+    return validate_shape(p, g, kHeadsSkip);
+}
+
 size_t plan_header_bytes(const Geometry &g)
 {
     return align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)g.heads + g.n_items), 256);

@@ -47,6 +47,8 @@ struct Geometry {
 // ----------------------------------------------------------- host-side helpers
 void set_error(const char *fmt, ...);
 svga_status validate_problem(const svga_problem *p, Geometry *g);
+// Shape checks and geometry only (per-head arrays not read).
+svga_status validate_geometry(const svga_problem *p, Geometry *g);
 size_t plan_header_bytes(const Geometry &g);  // header + head_info + items, 256-aligned
 int64_t plan_entry_cap(const Geometry &g);
 size_t align_up(size_t x, size_t a);

@@ -29,7 +29,7 @@ FLAG_TEST_STALL = 1 << 16
 EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",
             "svga_permute_tokens",
             "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_sparse_attention_fwd_part",
-            "svga_classify_heads_async", "svga_build_block_map_routed",
+            "svga_validate_block_map", "svga_classify_heads_async", "svga_build_block_map_routed",
             "svga_permute_tokens_mapped", "svga_unpermute_tokens_mapped",
             "svga_dense_attention_fwd",
             "svga_classify_size", "svga_classify_heads", "svga_last_error",
@@ -93,6 +93,7 @@ def load() -> ctypes.CDLL:
         lib.svga_build_block_map_routed.argtypes = [PP, P, P, P, ctypes.POINTER(BlockMapC), P,
                                                    SZ, P]
         lib.svga_permute_tokens_mapped.argtypes = [P, P, PP, ctypes.POINTER(BlockMapC), P]
+        lib.svga_validate_block_map.argtypes = [PP, ctypes.POINTER(BlockMapC), P]
         lib.svga_unpermute_tokens_mapped.argtypes = [P, P, PP, ctypes.POINTER(BlockMapC), P]
         lib.svga_last_error.restype = ctypes.c_char_p
         lib.svga_last_error.argtypes = []
@@ -205,6 +206,12 @@ def svga_build_block_map(problem: ProblemSpec, bmap: BlockMap, stream=None) -> B
 
 def build_block_map(problem: ProblemSpec, stream=None) -> BlockMap:
     return svga_build_block_map(problem, BlockMap(problem), stream)
+
+
+def svga_validate_block_map(problem: ProblemSpec, bmap: BlockMap, stream=None) -> None:
+    """Host-side consistency check of a built map; raises SvgaError naming the violation."""
+    _check(load().svga_validate_block_map(ctypes.byref(problem.c), ctypes.byref(bmap.c),
+                                          _stream(stream)))
 
 
 def svga_permute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,

@@ -190,6 +190,18 @@ SVGA_API svga_status svga_build_block_map(const svga_problem *problem, svga_bloc
 SVGA_API svga_status svga_build_block_map_static(const svga_problem *problem,
                                                  svga_block_map *map, svga_stream_t stream);
 
+/* Host-side consistency check of a built map, the stand-in for a race detector:
+ * copies the map to the host (synchronises `stream`) and checks that the status word
+ * is 0, classes are 0 / 1 / 2 and no tile holding padding is full, the CSR offsets
+ * start at 0, never decrease and fit the capacities, every list is strictly ascending,
+ * in range and agrees with the classes (complete, nothing extra), and the plan matches
+ * the problem: header, head info, one item per (head, query-block pair), items longest
+ * first, each item's entries exactly the visited key chunks in ascending order with
+ * visit / full flags recomputed from the classes.  Returns SVGA_OK, or
+ * SVGA_ERR_INVALID_ARG naming the first violation in svga_last_error. */
+SVGA_API svga_status svga_validate_block_map(const svga_problem *problem,
+                                             const svga_block_map *map, svga_stream_t stream);
+
 /* Token permutation of one tensor [heads, tokens, head_dim] bf16: for every head h,
  * dst[h, pos] = src[h, t] where pos is the position of frame-major token t in
  * order[h] (spatial heads usually stay frame-major: a plain copy).  The pages move

@@ -142,3 +142,53 @@ def test_plan_repacks_the_lists(wl, tq, tk):
             if a | b:
                 expect.append(c | (a << 24) | (b << 26))
         np.testing.assert_array_equal(ents, np.array(expect, np.uint32))
+
+
+# ------------------------------------------------- host-side map validator
+@pytest.mark.parametrize("wl,order,tq,tk", [
+    (C.tiny(), None, 64, 64),
+    (C.mid(), None, 128, 128),
+    (C.mid(), [C.ORDER_TEMPORAL_MAJOR_STRICT] * 4, 64, 256),
+    (C.mid(), [C.ORDER_FRAME_MAJOR] * 4, 256, 64),
+    (C.headline(), None, 128, 128),
+], ids=["tiny", "mid", "mid-strict-64x256", "mid-fm-256x64", "headline"])
+def test_validator_accepts_built_maps(wl, order, tq, tk):
+    prob = problem_of(wl, order, tq, tk)
+    bmap = svga.build_block_map(prob)
+    svga.svga_validate_block_map(prob, bmap)
+
+
+def _corrupted(what):
+    wl = C.mid()
+    prob = problem_of(wl, None, 128, 128)
+    bmap = svga.build_block_map(prob)
+    torch.cuda.synchronize()
+    if what == "class":           # a full tile turned boundary: lists no longer agree
+        k = int(torch.nonzero(bmap.cls == 1)[0].item())
+        bmap.cls[k] = 2
+    elif what == "order":         # two entries of a full list swapped
+        r = int(torch.nonzero(bmap.full_ptr[1:] - bmap.full_ptr[:-1] >= 2)[0].item())
+        a = int(bmap.full_ptr[r].item())
+        x, y = bmap.full_idx[a].item(), bmap.full_idx[a + 1].item()
+        bmap.full_idx[a], bmap.full_idx[a + 1] = y, x
+    elif what == "offset":        # a CSR offset decreasing
+        bmap.bnd_ptr[5] = bmap.bnd_ptr[4] - 1
+    elif what == "plan_flag":     # the full flag of a plan entry flipped
+        head = bmap.plan[:64].cpu().numpy().view(np.int32)
+        hdr = (64 + 16 * (int(head[1]) + int(head[11])) + 255) // 256 * 256
+        ent = bmap.plan[hdr:hdr + 4].view(torch.int32)
+        ent ^= 1 << 25
+    elif what == "status":
+        bmap.status.fill_(3)
+    torch.cuda.synchronize()
+    return prob, bmap
+
+
+@pytest.mark.parametrize("what,msg", [("class", "list"), ("order", "ascending"),
+                                      ("offset", "decrease"), ("plan_flag", "plan entry"),
+                                      ("status", "status word")])
+def test_validator_rejects_corrupted_maps(what, msg):
+    prob, bmap = _corrupted(what)
+    with pytest.raises(svga.SvgaError) as e:
+        svga.svga_validate_block_map(prob, bmap)
+    assert e.value.status == 1 and msg in str(e.value), str(e.value)
