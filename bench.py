@@ -200,6 +200,14 @@ def run_svga(args, rank, world, local_rank):
                            "order": order})
         classify = {"ms": classify_ms, "rows_per_head": n_rows, "types": list(types),
                     "mse": [[round(a, 9), round(b, 9)] for a, b in mse]}
+        if args.mode == "classify":
+            # profiling aid: the classifier alone (Q/K/V and its workspace on the device)
+            for _ in range(args.steps):
+                svga.svga_classify_heads(qd, kd, vd, prob0, wl.cand_spatial, wl.cand_temporal,
+                                         None, n_rows, scale, ws)
+            return {"study": "online head classification", "workload": wl.name, **classify}
+    elif args.mode == "classify":
+        raise SystemExit(f"{wl.name} has no classifier settings (use --config 2k)")
     prob = svga.ProblemSpec.from_workload(wl)
 
     # block map: built once (timed on its own)
@@ -533,7 +541,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--parts", type=int, default=8, help="number of parts for --mode parts")
-    ap.add_argument("--mode", default="full", choices=["full", "attn", "parts"],
+    ap.add_argument("--mode", default="full", choices=["full", "attn", "parts", "classify"],
                     help="attn: only launch the attention kernel (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

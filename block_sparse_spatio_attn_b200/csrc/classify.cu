@@ -9,8 +9,9 @@
 //   2. the tcgen05 attention kernel runs three times over all keys with the gathered
 //      rows as queries (their original coordinates ride along): dense, spatial-masked
 //      and temporal-masked, writing fp32 outputs;
-//   3. one block per head reduces the two squared deviations (fp64 accumulation) and
-//      picks the smaller one (a tie goes to spatial).
+//   3. the two squared deviations are reduced in fp64, first over slices of each head's
+//      outputs by many blocks, then per head in a fixed order (deterministic), and the
+//      smaller one picks the mask (a tie goes to spatial).
 #include <cuda_runtime.h>
 
 #include "svga_device.cuh"
@@ -56,14 +57,19 @@ __global__ void gather_rows_kernel(const uint4 *__restrict__ q, uint4 *__restric
     }
 }
 
-__global__ void __launch_bounds__(256) mse_kernel(const float *od, const float *os, const float *ot,
-                                                  int n, int32_t *type_out, float *mse_out)
+constexpr int kMseParts = 32;  // blocks per head in the first reduction stage
+
+// Stage 1: block (part, h) sums the squared deviations of one slice of head h.
+__global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const float *os,
+                                                          const float *ot, int n, double *partial)
 {
     __shared__ double red[2][8];
-    const int h = blockIdx.x;
+    const int part = blockIdx.x, h = blockIdx.y;
     const size_t base = (size_t)h * n;
+    const int per = (n + kMseParts - 1) / kMseParts;
+    const int i0 = part * per, i1 = min(n, i0 + per);
     double as = 0.0, at = 0.0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
         const double d = od[base + i];
         const double a = os[base + i] - d, b = ot[base + i] - d;
         as += a * a;
@@ -84,16 +90,31 @@ __global__ void __launch_bounds__(256) mse_kernel(const float *od, const float *
             s += red[0][w];
             t += red[1][w];
         }
-        s /= n;
-        t /= n;
-        mse_out[2 * h] = (float)s;
-        mse_out[2 * h + 1] = (float)t;
-        type_out[h] = s <= t ? MASK_SPATIAL : MASK_TEMPORAL;
+        partial[((size_t)h * kMseParts + part) * 2] = s;
+        partial[((size_t)h * kMseParts + part) * 2 + 1] = t;
     }
 }
 
+// Stage 2: per head, the partial sums in part order, the means and the decision.
+__global__ void mse_final_kernel(const double *partial, int heads, int n, int32_t *type_out,
+                                 float *mse_out)
+{
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= heads) return;
+    double s = 0.0, t = 0.0;
+    for (int part = 0; part < kMseParts; ++part) {
+        s += partial[((size_t)h * kMseParts + part) * 2];
+        t += partial[((size_t)h * kMseParts + part) * 2 + 1];
+    }
+    s /= n;
+    t /= n;
+    mse_out[2 * h] = (float)s;
+    mse_out[2 * h + 1] = (float)t;
+    type_out[h] = s <= t ? MASK_SPATIAL : MASK_TEMPORAL;
+}
+
 struct ClassifyLayout {
-    size_t info_s, info_t, rows, qg, od, os, ot, types, mse, status, total;
+    size_t info_s, info_t, rows, qg, od, os, ot, partial, types, mse, status, total;
 };
 
 ClassifyLayout classify_layout(int heads, int d, int n_rows)
@@ -112,6 +133,7 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows)
     L.od = take((size_t)heads * n_rows * d * 4);
     L.os = take((size_t)heads * n_rows * d * 4);
     L.ot = take((size_t)heads * n_rows * d * 4);
+    L.partial = take(sizeof(double) * 2 * kMseParts * heads);
     L.types = take(sizeof(int32_t) * heads);
     L.mse = take(sizeof(float) * 2 * heads);
     L.status = take(sizeof(int32_t));
@@ -206,7 +228,9 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.head_info = reinterpret_cast<const int32_t *>(info_t);
     a.o = ot;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
-    mse_kernel<<<H, 256, 0, st>>>(od, os, ot, n_rows * d, types, mse);
+    double *partial = reinterpret_cast<double *>(w + L.partial);
+    mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(od, os, ot, n_rows * d, partial);
+    mse_final_kernel<<<(H + 127) / 128, 128, 0, st>>>(partial, H, n_rows * d, types, mse);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("classifier reduction launch failed: %s", cudaGetErrorString(e));
