@@ -62,6 +62,8 @@ struct KParams {
     int mode, naive, aligned, n_pairs, n_qblk, n_kc;
     int n_items, part, num_parts;  // plan mode: this launch runs the items of one part
     int test_stall;                // test hook: the first K chunk is never loaded
+    int qo_fm;                     // Q and O frame-major: Q rows gathered, O rows scattered
+    const void *q;                 // Q base (for the gather)
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Item it = make_item(p, KN);
 
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bar->q_full), 1);
+        mbar_init(smem_u32(&bar->q_full), p.qo_fm ? 8 : 1);  // 8 gathering warps, or TMA
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&bar->kv_full[s]), 1);
             mbar_init(smem_u32(&bar->kv_empty[s]), 1);
@@ -309,11 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             const uint32_t qf = smem_u32(&bar->q_full);
-            mbar_arrive_expect_tx(qf, (it.valid1 ? 2 : 1) * C::kQBytes);
-            for (int i = 0; i < (it.valid1 ? 2 : 1); ++i)
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(smem_u32(sQ + i * C::kQBytes + c * C::kQChunk), &tmQ, qf, 64 * c,
-                                (it.b0 + i) * kBlockM, it.h);
+            if (!p.qo_fm) {
+                mbar_arrive_expect_tx(qf, (it.valid1 ? 2 : 1) * C::kQBytes);
+                for (int i = 0; i < (it.valid1 ? 2 : 1); ++i)
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(smem_u32(sQ + i * C::kQBytes + c * C::kQChunk), &tmQ, qf,
+                                    64 * c, (it.b0 + i) * kBlockM, it.h);
+            }
             int issued = 0;
             bool ok = true;
             for (int n = 0; n < it.E && ok; ++n) {
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) {
                 // Abort: let the copies in flight land before the CTA exits.
-                mbar_wait_bounded(qf, 0);
+                if (!p.qo_fm) mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
                     if (!(p.test_stall && idx == 0))
                         mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
@@ -466,6 +470,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pos_to_coord(korder, qpos, p.F, p.S, fq, sq);
             }
         }
+        // Q and O frame-major: each thread copies its own Q row from the row's frame-major
+        // token into the 128-byte-swizzled Q tile (the layout the TMA load would give),
+        // and O / LSE go back to that token.
+        int tok = qpos;
+        if (p.qo_fm) {
+            if (row_valid) tok = fq * p.S + sq;
+            const uint32_t qs = smem_u32(sQ + wg * C::kQBytes) + row * 128;
+            const uint4 *src = static_cast<const uint4 *>(p.q) +
+                               ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * (D / 8);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 x = row_valid ? __ldg(src + c * 8 + u) : make_uint4(0, 0, 0, 0);
+                    st_shared_v4(qs + c * C::kQChunk + ((u ^ (row & 7)) << 4), x.x, x.y, x.z,
+                                 x.w);
+                }
+            fence_proxy_async_smem();  // generic-proxy stores -> visible to the MMA
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar->q_full));
+        }
         const uint32_t vbit = wg ? kEntV1 : kEntV0, fbit = wg ? kEntF1 : kEntF0;
         const float sl2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
@@ -585,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && (blk < p.n_qblk)) {
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t orow = ((size_t)it.h * p.nq_rows + (row_valid ? qpos : 0)) * D;
+            const size_t orow = ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * D;
 #pragma unroll 1
             for (int j = 0; j < D / 32; ++j) {
                 uint32_t o[32];
@@ -623,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (row_valid && p.lse)
-                p.lse[(size_t)it.h * p.nq_rows + qpos] =
+                p.lse[(size_t)it.h * p.nq_rows + tok] =
                     l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
     }
@@ -732,6 +757,8 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.part = a.part;
     kp.num_parts = a.num_parts > 0 ? a.num_parts : 1;
     kp.test_stall = a.test_stall;
+    kp.qo_fm = a.qo_fm;
+    kp.q = a.q;
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;

@@ -82,6 +82,7 @@ struct AttnLaunch {
     int aligned;               // plan mode: keep every key of a visited tile (mask snapped to tiles)
     int part, num_parts;       // plan mode: run only the items of part `part` (0 of 1: all)
     int test_stall;            // SVGA_FLAG_TEST_STALL: withhold the first K load
+    int qo_fm;                 // SVGA_FLAG_QO_FRAME_MAJOR: q, o, lse frame-major
     int kn;                    // keys per chunk: 64 or 128
     const void *plan;          // device plan (mode 0)
     const int32_t *head_info;  // device int4 per head (modes 0 and 2)

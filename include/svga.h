@@ -86,6 +86,13 @@ enum {
      * plain masked softmax over that set.  Needs tile_q >= 128 (SVGA_ERR_UNSUPPORTED
      * otherwise); cannot be combined with SVGA_FLAG_NAIVE_B1 (SVGA_ERR_INVALID_ARG). */
     SVGA_FLAG_TILE_ALIGNED = 2,
+    /* q, o and lse are FRAME-MAJOR for every head (k and v stay in order[h]): the
+     * kernel gathers each query row from its frame-major token and writes O and LSE
+     * back to it, so the permutation of Q and the inverse permutation of O are not
+     * needed (the pages move the tokens of temporal heads to temporal-major order,
+     * ainews.tenesys.com, "Co sie zmienilo?" item 5; here only K and V move).
+     * Results are identical bit for bit to permute -> attention -> unpermute. */
+    SVGA_FLAG_QO_FRAME_MAJOR = 4,
     /* Test hook for the failure path: the first K chunk of every CTA is never loaded,
      * so the kernel's bounded waits run out (about one second per CTA wave), every role
      * stops, copies in flight are drained, TMEM is released and map->status reads

@@ -231,7 +231,7 @@ def test_tile_aligned_flag_validation():
     with pytest.raises(svga.SvgaError) as e:
         run_sparse_path(wl, qd, kd, vd, tile_q=64, tile_k=128, flags=svga.FLAG_TILE_ALIGNED)
     assert e.value.status == 4
-    for bad in (svga.FLAG_TILE_ALIGNED | svga.FLAG_NAIVE_B1, 4):
+    for bad in (svga.FLAG_TILE_ALIGNED | svga.FLAG_NAIVE_B1, 1 << 8):   # unknown bit
         with pytest.raises(svga.SvgaError) as e:
             run_sparse_path(wl, qd, kd, vd, flags=bad)
         assert e.value.status == 1
@@ -298,3 +298,33 @@ def test_part_argument_checks():
         with pytest.raises(svga.SvgaError) as e:
             svga.svga_sparse_attention_fwd_part(qd, kd, vd, o, None, prob, bmap, 0.125, 0, part, n)
         assert e.value.status == 1
+
+
+# ------------------------------- Q and O frame-major (only K and V permuted)
+@pytest.mark.parametrize("name,flags,tiles", [
+    ("tiny", 0, None), ("mid", 0, None), ("mid", svga.FLAG_NAIVE_B1, None),
+    ("mid", svga.FLAG_TILE_ALIGNED, (256, 128)), ("mid", 0, (64, 64)), ("headline", 0, None)])
+def test_qo_frame_major_equals_permuted_path(name, flags, tiles):
+    """The kernel's own gather of Q rows and scatter of O rows gives the same bits as
+    permute(Q) -> attention -> unpermute(O), and LSE lands at the frame-major token."""
+    wl = C.ALL[name]()
+    if tiles:
+        wl = wl.with_tile(*tiles)
+    q, k, v, qd, kd, vd = inputs(wl)
+    o_ref, lse_ref, _ = run_sparse_path(wl, qd, kd, vd, flags=flags)
+    lse_ref = lse_to_frame_major(lse_ref.cpu().numpy(), wl, wl.order)
+    prob = svga.ProblemSpec.from_workload(wl)
+    bmap = svga.build_block_map(prob)
+    kp, vp = torch.empty_like(kd), torch.empty_like(vd)
+    svga.svga_permute_tokens(kd, kp, prob)
+    svga.svga_permute_tokens(vd, vp, prob)
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.empty(wl.heads, wl.tokens, dtype=torch.float32, device="cuda")
+    for part in range(2):   # two parts: each writes only its own rows, together all rows
+        svga.svga_sparse_attention_fwd_part(qd, kp, vp, o, lse, prob, bmap,
+                                            1.0 / math.sqrt(wl.head_dim),
+                                            flags | svga.FLAG_QO_FRAME_MAJOR, part, 2)
+    torch.cuda.synchronize()
+    assert bmap.device_status() == 0
+    assert torch.equal(o, o_ref)
+    np.testing.assert_array_equal(lse.cpu().numpy(), lse_ref)
