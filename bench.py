@@ -87,6 +87,12 @@ def weak_scaling_value(flops_per_rank: float, world: int, ms_per_step: float) ->
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
+def job_value(flops_per_problem: float, world: int, ms_per_step: float, split: bool) -> float:
+    """TFLOP/s of the whole job: with `split` the ranks share one problem (strong
+    scaling), otherwise every rank runs its own (weak scaling)."""
+    return weak_scaling_value(flops_per_problem, 1 if split else world, ms_per_step)
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -168,6 +174,8 @@ def run_svga(args, rank, world, local_rank):
     from block_sparse_spatio_attn_b200 import svga
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    split = bool(args.split) and world > 1
+    part, n_parts = (rank, world) if split else (0, 1)
     wl = C.ALL[args.config]()
     if args.tile:
         tq, tk = (int(x) for x in args.tile.lower().split("x"))
@@ -237,8 +245,8 @@ def run_svga(args, rank, world, local_rank):
         svga.svga_permute_tokens(vd, vp, prob)
         if attn_evs is not None:
             attn_evs[0].record(stream)
-        svga.svga_sparse_attention_fwd(qd, kp, vp, o, None, prob, bmap, scale,
-                                       svga.FLAG_QO_FRAME_MAJOR)
+        svga.svga_sparse_attention_fwd_part(qd, kp, vp, o, None, prob, bmap, scale,
+                                            svga.FLAG_QO_FRAME_MAJOR, part, n_parts)
         if attn_evs is not None:
             attn_evs[1].record(stream)
 
@@ -378,8 +386,8 @@ def run_svga(args, rank, world, local_rank):
         bq, bk, bv, bqp, bkp, bvp, bop, bo = bs
         svga.svga_permute_tokens(bk, bkp, prob)
         svga.svga_permute_tokens(bv, bvp, prob)
-        svga.svga_sparse_attention_fwd(bq, bkp, bvp, bo, None, prob, bmap, scale,
-                                       svga.FLAG_QO_FRAME_MAJOR)
+        svga.svga_sparse_attention_fwd_part(bq, bkp, bvp, bo, None, prob, bmap, scale,
+                                            svga.FLAG_QO_FRAME_MAJOR, part, n_parts)
 
     def e2e_run(n, t0=None, t1=None):
         for i in range(n):
@@ -421,22 +429,25 @@ def run_svga(args, rank, world, local_rank):
     timed_s = elapsed / 1e3
     sustained = timed_s >= 2.0
     peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    achieved = visited_flops / (attn_ms * 1e-3) / 1e12
+    launch_flops = visited_flops / n_parts   # split: about 1/n of the items per rank
+    achieved = launch_flops / (attn_ms * 1e-3) / 1e12
     traffic = traffic_from_profile(os.path.join(ROOT, "block_sparse_spatio_attn_b200", "csrc",
                                                 "attention.cu"))
     if traffic is not None and args.config != "headline":
         traffic = None
     out = {
-        "metric": METRIC, "value": weak_scaling_value(kflops, world, ms_per_step),
+        "metric": METRIC, "value": job_value(kflops, world, ms_per_step, split),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "tokens": N, "heads": H, "head_dim": d,
                    "frames": wl.frames, "grid": f"{wl.grid_h}x{wl.grid_w}",
                    "head_types": "".join("ST"[t] for t in wl.head_type), "bands": wl.band,
                    "orders": wl.order, "tile": f"{wl.tile_q}x{wl.tile_k}",
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "parallelism": (f"parts{world}" if split else f"replicas{world}")
+                   if world > 1 else "single",
                    "l2": "inputs larger than L2 (Q,K,V %.0f MB)" % (3 * H * N * d * 2 / 1e6),
                    "step": "permute K,V + sparse attention (Q rows gathered and O rows "
                            "written frame-major by the kernel)"},
@@ -453,8 +464,8 @@ def run_svga(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} {'sustained' if sustained else 'burst'} bf16",
-                     "kernel": "attn_fwd_kernel<128,128>", "flops_per_launch": visited_flops},
-        "e2e": {"value": weak_scaling_value(kflops, world, e2e_ms), "unit": "TFLOP/s",
+                     "kernel": "attn_fwd_kernel<128,128>", "flops_per_launch": launch_flops},
+        "e2e": {"value": job_value(kflops, world, e2e_ms, split), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * H * N * d * 2,
                 "d2h_bytes_per_step": H * N * d * 2,
                 "pipeline": "copy-in, compute and copy-out of successive steps overlap on "
@@ -555,6 +566,9 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--parts", type=int, default=8, help="number of parts for --mode parts")
+    ap.add_argument("--split", action="store_true",
+                    help="under torchrun, the ranks share one problem (each runs its part of "
+                         "the work items) instead of running one problem each")
     ap.add_argument("--mode", default="full", choices=["full", "attn", "parts", "classify"],
                     help="attn: only launch the attention kernel (for ncu captures)")
     args = ap.parse_args()

@@ -46,6 +46,14 @@ def test_weak_scaling_value_and_single_process_identity():
     assert bench.max_over_ranks([3.0, 4.0], torch.device("cpu")) == [3.0, 4.0]
 
 
+def test_job_value_weak_and_strong():
+    import bench
+    # replicas: every rank its own problem; split: the ranks share one problem
+    assert abs(bench.job_value(1e13, 4, 10.0, split=False) - 4000.0) < 1e-9
+    assert abs(bench.job_value(1e13, 4, 2.5, split=True) - 4000.0) < 1e-9
+    assert bench.job_value(1e13, 1, 10.0, True) == bench.job_value(1e13, 1, 10.0, False)
+
+
 def test_closed_form_kept_pairs_match_the_oracle():
     """bench.py's FLOP accounting (closed form per head and per row) equals the oracle's
     pair counts."""
