@@ -328,3 +328,10 @@ def test_qo_frame_major_equals_permuted_path(name, flags, tiles):
     assert bmap.device_status() == 0
     assert torch.equal(o, o_ref)
     np.testing.assert_array_equal(lse.cpu().numpy(), lse_ref)
+    if name == "headline" and flags == 0:
+        # the launch the bench times, checked against the oracle directly as well
+        rows = sample_rows(wl, 96)
+        on, ln = o.float().cpu().numpy(), lse.cpu().numpy()
+        for h in (0, wl.heads - 1):          # one spatial and one temporal head
+            ro, rl = oracle_rows(wl, q, k, v, h, rows)
+            assert_attn_close(on[h, rows], ro, ln[h, rows], rl, what=f"headline QO-FM head {h}")
