@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Item it = make_item(p, KN);
 
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bar->q_full), p.qo_fm ? 8 : 1);  // 8 gathering warps, or TMA
+        mbar_init(smem_u32(&bar->q_full), 1);  // the TMA load, or the last gathering warp
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&bar->kv_full[s]), 1);
             mbar_init(smem_u32(&bar->kv_empty[s]), 1);
@@ -311,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             const uint32_t qf = smem_u32(&bar->q_full);
-            if (!p.qo_fm) {
+            // frame-major Q of a head in frame-major order is already in the head's order
+            const bool q_tma = !p.qo_fm || __ldg(p.head_info + it.h).z == ORDER_FM;
+            if (q_tma) {
                 mbar_arrive_expect_tx(qf, (it.valid1 ? 2 : 1) * C::kQBytes);
                 for (int i = 0; i < (it.valid1 ? 2 : 1); ++i)
                     for (int c = 0; c < D / 64; ++c)
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) {
                 // Abort: let the copies in flight land before the CTA exits.
-                if (!p.qo_fm) mbar_wait_bounded(qf, 0);
+                if (q_tma) mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
                     if (!(p.test_stall && idx == 0))
                         mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
@@ -474,8 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // token into the 128-byte-swizzled Q tile (the layout the TMA load would give),
         // and O / LSE go back to that token.
         int tok = qpos;
-        if (p.qo_fm) {
-            if (row_valid) tok = fq * p.S + sq;
+        if (p.qo_fm && row_valid) tok = fq * p.S + sq;
+        if (p.qo_fm && korder != ORDER_FM) {
             const uint32_t qs = smem_u32(sQ + wg * C::kQBytes) + row * 128;
             const uint4 *src = static_cast<const uint4 *>(p.q) +
                                ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * (D / 8);
@@ -488,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  x.w);
                 }
             fence_proxy_async_smem();  // generic-proxy stores -> visible to the MMA
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bar->q_full));
+            named_bar_sync(1, 256);    // both groups' rows are in place
+            if (warp == 4 && lane == 0) mbar_arrive(smem_u32(&bar->q_full));
         }
         const uint32_t vbit = wg ? kEntV1 : kEntV0, fbit = wg ? kEntF1 : kEntF0;
         const float sl2 = p.scale_log2;
