@@ -27,7 +27,10 @@
 //   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated);
 //   * a launch may run one part of the plan's items (snake order), so one problem can
 //     be split over several GPUs; the tile-aligned traversal (B3) treats every visited
-//     chunk as full.
+//     chunk as full;
+//   * with Q and O frame-major, the softmax threads of a temporal-major head copy their
+//     own Q rows into the swizzled Q tile (frame-major heads keep the TMA load) and
+//     every head writes O and LSE rows back to their frame-major tokens.
 //
 // Every mbarrier wait gives up after about a second: the CTA raises a shared abort
 // flag, drains its MMAs and copies, frees TMEM, writes SVGA_ERR_TIMEOUT to the
