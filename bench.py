@@ -2,15 +2,21 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl svga|reference]
                     [--config headline|mid|tiny|permstudy|2k] [--tile 128x128]
+                    [--order fm|tm|strict] [--split] [--mode full|attn|parts|classify]
 
-One step = one pass of the hot path over the workload's Q/K/V already in HBM:
-token permutation of Q, K, V into each head's order, block-sparse attention, inverse
-permutation of O.  The block map depends on the problem only and is built once before
+One step = one pass of the hot path over the workload's Q/K/V already in HBM: K and V
+permuted into each head's token order, then the block-sparse attention, which takes Q
+frame-major (gathering the rows of temporal-major heads itself) and writes O
+frame-major; the same step with Q permuted and O unpermuted by separate kernels is
+timed beside it.  The block map depends on the problem only and is built once before
 timing (its build time is reported separately), as it would be cached across layers and
 denoising steps.  Metric: effective TFLOP/s on kept pairs, FLOP = sum over heads of
 4 * kept_pairs * head_dim, and ms per step.  Under torchrun every rank runs the same
-workload on its own GPU (weak scaling); value = FLOP of all ranks / max time over ranks.
+workload on its own GPU (weak scaling; value = FLOP of all ranks / max time over ranks),
+or with --split the ranks share one problem (strong scaling).
 
+--mode attn / classify only launch the attention kernel / the classifier (for ncu
+captures); --mode parts times each part of a split problem alone.
 --impl reference times the fp64 CPU oracle (the only reference this method has) on a
 bounded sample of query rows per step, on rank 0 only.
 """
