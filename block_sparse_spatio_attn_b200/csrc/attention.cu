@@ -523,22 +523,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 keep_mask<KN>(korder, p.aligned ? MASK_DENSE : type, band, p.anchor, p.F, p.S,
                               p.nk_rows, fq, sq, kc * KN, keep);
             tmem_wait_ld();
-            // A masked chunk that every row of this warp keeps whole, or drops whole, needs
-            // no per-element select: the first runs the unmasked body, the second only
-            // stores P = 0 (the row maximum and sum do not change).  Same bits either way.
-            int path = full ? 0 : 1;  // 0 unmasked, 1 masked, 2 nothing kept
-            if (!full) {
-                uint32_t all = 0xFFFFFFFFu, any = 0u;
-#pragma unroll
-                for (int w = 0; w < KN / 32; ++w) {
-                    all &= keep[w];
-                    any |= keep[w];
-                }
-                if (__all_sync(0xffffffffu, all == 0xFFFFFFFFu))
-                    path = 0;
-                else if (__all_sync(0xffffffffu, any == 0u))
-                    path = 2;
-            }
 
             // The two instantiations: full tiles carry no mask arithmetic.
             auto body = [&](auto masked_tag) {
@@ -610,17 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 l += (s0.x + s0.y) + (s1.x + s1.y);
             };
-            if (path == 0) {
+            if (full)
                 body(std::false_type{});
-            } else if (path == 1) {
+            else
                 body(std::true_type{});
-            } else {
-                uint32_t zero[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) zero[c] = 0u;
-#pragma unroll
-                for (int j = 0; j < KN / 32; ++j) tmem_st16(tS + j * 16, zero);
-            }
             if (!ok) break;
             tmem_wait_st();
             // every lane's P is in TMEM (wait::st + fence); after the warp-level sync one
