@@ -231,10 +231,14 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  * element (aihirek.info, section "A TPU-kernel kialakitasa ...").  An empty row
  * gives O = 0 and lse = -inf.
  *   q, k, v, o : DEVICE bf16 [heads, tokens, head_dim], every head in order[h]
- *   lse        : DEVICE float [heads, tokens] or NULL
- *   map        : built by svga_build_block_map for this same problem
+ *                (q and o frame-major instead with SVGA_FLAG_QO_FRAME_MAJOR)
+ *   lse        : DEVICE float [heads, tokens] or NULL (frame-major with that flag)
+ *   map        : built by svga_build_block_map (or _routed / _static) for this problem;
+ *                the per-head type, band and order are read from the map's plan
  *   scale      : softmax scale, usually 1/sqrt(head_dim)
- *   flags      : 0, SVGA_FLAG_NAIVE_B1 or SVGA_FLAG_TILE_ALIGNED
+ *   flags      : 0 or a combination of SVGA_FLAG_NAIVE_B1 / SVGA_FLAG_TILE_ALIGNED
+ *                (not both), SVGA_FLAG_QO_FRAME_MAJOR and the test hook
+ *                SVGA_FLAG_TEST_STALL; other bits give SVGA_ERR_INVALID_ARG
  * bf16 inputs, fp32 accumulation and softmax, P rounded to bf16 for the PV product. */
 SVGA_API svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,
                                       float *lse, const svga_problem *problem,
