@@ -335,3 +335,28 @@ def test_qo_frame_major_equals_permuted_path(name, flags, tiles):
         for h in (0, wl.heads - 1):          # one spatial and one temporal head
             ro, rl = oracle_rows(wl, q, k, v, h, rows)
             assert_attn_close(on[h, rows], ro, ln[h, rows], rl, what=f"headline QO-FM head {h}")
+
+
+def test_maximum_head_count():
+    """4,096 heads (the largest count the library takes), 2 frames of 4x6 tokens, d = 64:
+    the per-head parameters travel as kernel parameters sized for that many heads.
+    Block map, permutation, attention and classification run for every head; a sample
+    of heads is checked against the oracle."""
+    H = 4096
+    types = [C.SPATIAL if h % 2 == 0 else C.TEMPORAL for h in range(H)]
+    wl = C.Workload("maxheads", 2, 4, 6, 64, types, [0 if t == C.SPATIAL else 5 for t in types],
+                    [C.ORDER_FRAME_MAJOR if t == C.SPATIAL else C.ORDER_TEMPORAL_MAJOR
+                     for t in types], seed=13)
+    q, k, v, qd, kd, vd = inputs(wl)
+    o, lse, bmap = run_sparse_path(wl, qd, kd, vd)
+    svga.svga_validate_block_map(svga.ProblemSpec.from_workload(wl), bmap)
+    o = o.float().cpu().numpy()
+    lse = lse_to_frame_major(lse.cpu().numpy(), wl, wl.order)
+    rows = np.arange(wl.tokens, dtype=np.int32)
+    for h in (0, 1, 2047, 4094, 4095):
+        ro, rl = oracle_rows(wl, q, k, v, h, rows)
+        assert_attn_close(o[h], ro, lse[h], rl, what=f"maxheads head {h}")
+    prob = svga.ProblemSpec.from_workload(wl)
+    t, _ = svga.svga_classify_heads(qd, kd, vd, prob, [1] * H, [3] * H, None, 8,
+                                    1.0 / math.sqrt(64))
+    assert len(t) == H and set(t) <= {0, 1}
