@@ -6,9 +6,13 @@
 // Video Diffusion on TPUs", aihirek.info, section "A Sparse VideoGen a figyelmi
 // fejeket osztalyozza").  Here:
 //   1. the sampled rows of Q are gathered into a compact [heads, n_rows, d] tensor;
-//   2. the tcgen05 attention kernel runs three times over all keys with the gathered
-//      rows as queries (their original coordinates ride along): dense, spatial-masked
-//      and temporal-masked, writing fp32 outputs;
+//   2. the tcgen05 attention kernel runs three times with the gathered rows as queries
+//      (their original coordinates ride along), writing fp32 outputs: dense over all
+//      keys, then spatial-masked and temporal-masked through small plans of their own:
+//      each 128-row block of sampled rows is bounded by the min / max of its rows'
+//      frame and in-frame index, which decides per key chunk whether it can hold a kept
+//      pair (conservative) and whether every pair is kept (exact), so that the masked
+//      passes skip empty chunks and run full ones unmasked;
 //   3. the two squared deviations are reduced in fp64, first over slices of each head's
 //      outputs by many blocks, then per head in a fixed order (deterministic), and the
 //      smaller one picks the mask (a tie goes to spatial).
@@ -60,6 +64,187 @@ __global__ void gather_rows_kernel(const uint4 *__restrict__ q, uint4 *__restric
 constexpr int kMseParts = 32;  // blocks per head in the first reduction stage
 
 // Stage 1: block (part, h) sums the squared deviations of one slice of head h.
+// Frame and in-frame index bounds (min f, max f, min s, max s) of each 128-row block of
+// sampled rows.  Rows outside 0..N-1 are clamped here (the gather reports them).
+__global__ void __launch_bounds__(128) row_bounds_kernel(const int32_t *rows, int n_rows, int N,
+                                                         int S, int4 *bounds)
+{
+    __shared__ int red[4][4];
+    const int r = blockIdx.x * 128 + threadIdx.x;
+    int fmin = 0x7fffffff, fmax = -1, smin = 0x7fffffff, smax = -1;
+    if (r < n_rows) {
+        int t = __ldg(rows + r);
+        t = t < 0 ? 0 : (t >= N ? N - 1 : t);
+        const int f = t / S, s = t - f * S;
+        fmin = fmax = f;
+        smin = smax = s;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
+        fmax = max(fmax, __shfl_xor_sync(0xffffffffu, fmax, o));
+        smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+        smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    }
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        red[w][0] = fmin;
+        red[w][1] = fmax;
+        red[w][2] = smin;
+        red[w][3] = smax;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < 4; ++i) {
+            fmin = min(fmin, red[i][0]);
+            fmax = max(fmax, red[i][1]);
+            smin = min(smin, red[i][2]);
+            smax = max(smax, red[i][3]);
+        }
+        bounds[blockIdx.x] = make_int4(fmin, fmax, smin, smax);
+    }
+}
+
+// Visit / full flags (1 | 2) of key chunk c (128 frame-major keys) for a block of rows
+// with bounds bb, under a mask of `type` and `band`.  A chunk is at most three
+// rectangles (frame x in-frame range): the first partial frame, whole frames, the last
+// partial frame; only the first can be frame 0.  "Visit" from the distance between the
+// bound intervals is a superset of the chunks that hold kept pairs; "full" compares the
+// farthest pair, which is exact.
+__device__ uint32_t chunk_flags(int4 bb, int type, int band, int anchor, int c, int N, int S)
+{
+    if (bb.y < 0) return 0u;
+    const int ka = c * 128, kb = min(N, ka + 128);
+    const int F0 = ka / S, m0 = ka - F0 * S, F1 = (kb - 1) / S, m1 = (kb - 1) - F1 * S;
+    bool any = false, all = ka + 128 <= N;  // a chunk holding padding is never full
+    auto rect = [&](int f0, int f1, int s0, int s1) {
+        const bool anch = anchor && f0 == 0;
+        int dist, far;
+        if (type == MASK_SPATIAL) {
+            dist = max(0, max(f0 - bb.y, bb.x - f1));
+            far = max(bb.y - f0, f1 - bb.x);
+        } else {
+            dist = max(0, max(s0 - bb.w, bb.z - s1));
+            far = max(bb.w - s0, s1 - bb.z);
+        }
+        any = any || anch || dist <= band;
+        all = all && (anch || far <= band);
+    };
+    if (F0 == F1) {
+        rect(F0, F0, m0, m1);
+    } else {
+        rect(F0, F0, m0, S - 1);
+        if (F1 > F0 + 1) rect(F0 + 1, F1 - 1, 0, S - 1);
+        rect(F1, F1, 0, m1);
+    }
+    return any ? (1u | (all ? 2u : 0u)) : 0u;
+}
+
+// The attention plan's entry for work item (head info hi, row-block pair p) and chunk c.
+__device__ __forceinline__ uint32_t pass_entry(const int4 &hi, int anchor, const int4 *bounds,
+                                               int n_qblk, int p, int c, int N, int S)
+{
+    const uint32_t a =
+        2 * p < n_qblk ? chunk_flags(bounds[2 * p], hi.x, hi.y, anchor, c, N, S) : 0u;
+    const uint32_t b =
+        2 * p + 1 < n_qblk ? chunk_flags(bounds[2 * p + 1], hi.x, hi.y, anchor, c, N, S) : 0u;
+    if (!(a | b)) return 0u;
+    return (uint32_t)c | (a << 24) | (b << 26);
+}
+
+// Entries per work item (a head and two row blocks) of one pass plan.
+__global__ void __launch_bounds__(256) pass_count_kernel(int n_pairs, int n_qblk, int n_kc, int N,
+                                                         int S, int anchor, const int4 *head_info,
+                                                         const int4 *bounds, int *cnt)
+{
+    __shared__ int red[8];
+    const int item = blockIdx.x, h = item / n_pairs, p = item - h * n_pairs;
+    const int4 hi = head_info[h];
+    int n = 0;
+    for (int c = threadIdx.x; c < n_kc; c += blockDim.x)
+        n += pass_entry(hi, anchor, bounds, n_qblk, p, c, N, S) != 0u;
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = n;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        cnt[item] = t;
+    }
+}
+
+// Exclusive offsets of the items' entries, the items and the plan header (one block).
+__global__ void __launch_bounds__(1024) pass_items_kernel(int heads, int n_pairs, int n_items,
+                                                          int N, int n_kc, const int *cnt,
+                                                          int *off, int4 *items, char *plan)
+{
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int base = 0; base < n_items; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < n_items ? cnt[i] : 0;
+        int x = v;  // inclusive scan inside the warp
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        int before = carry;
+        for (int j = 0; j < w; ++j) before += wsum[j];
+        if (i < n_items) {
+            const int start = before + x - v;
+            off[i] = start;
+            const int h = i / n_pairs, p = i - h * n_pairs;
+            items[i] = make_int4(h, 2 * p, start, v);
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = before + x;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        PlanHeader hdr{};
+        hdr.magic = kPlanMagic;
+        hdr.heads = heads;
+        hdr.tokens = N;
+        hdr.kn = 128;
+        hdr.n_kc = n_kc;
+        hdr.n_items = n_items;
+        *reinterpret_cast<PlanHeader *>(plan) = hdr;
+    }
+}
+
+// The entries of each item, in ascending chunk order.
+__global__ void __launch_bounds__(128) pass_write_kernel(int n_pairs, int n_qblk, int n_kc, int N,
+                                                         int S, int anchor, const int4 *head_info,
+                                                         const int4 *bounds, const int *off,
+                                                         uint32_t *entries)
+{
+    __shared__ int wsum[4];
+    const int item = blockIdx.x, h = item / n_pairs, p = item - h * n_pairs;
+    const int4 hi = head_info[h];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int o = off[item];
+    for (int base = 0; base < n_kc; base += 128) {
+        const int c = base + threadIdx.x;
+        const uint32_t e = c < n_kc ? pass_entry(hi, anchor, bounds, n_qblk, p, c, N, S) : 0u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, e != 0u);
+        const int pos = __popc(bal & ((1u << lane) - 1u));
+        if (lane == 0) wsum[w] = __popc(bal);
+        __syncthreads();
+        int before = 0, tot = 0;
+        for (int i = 0; i < 4; ++i) {
+            before += i < w ? wsum[i] : 0;
+            tot += wsum[i];
+        }
+        if (e != 0u) entries[o + before + pos] = e;
+        o += tot;
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const float *os,
                                                           const float *ot, int n, double *partial)
 {
@@ -114,10 +299,11 @@ __global__ void mse_final_kernel(const double *partial, int heads, int n, int32_
 }
 
 struct ClassifyLayout {
-    size_t info_s, info_t, rows, qg, od, os, ot, partial, types, mse, status, total;
+    size_t plan_s, plan_t, plan_hdr, bounds, cnt, off, rows, qg, od, os, ot, partial, types, mse,
+        status, total;
 };
 
-ClassifyLayout classify_layout(int heads, int d, int n_rows)
+ClassifyLayout classify_layout(int heads, int d, int n_rows, int N)
 {
     ClassifyLayout L{};
     size_t o = 0;
@@ -126,8 +312,16 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows)
         o = align_up(o + bytes, 256);
         return at;
     };
-    L.info_s = take(sizeof(int4) * heads);
-    L.info_t = take(sizeof(int4) * heads);
+    // the two pass plans, in the attention plan's layout
+    const int n_qblk = (n_rows + kBlockM - 1) / kBlockM, n_items = heads * ((n_qblk + 1) / 2);
+    const int n_kc = (N + 127) / 128;
+    L.plan_hdr = align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)heads + n_items), 256);
+    const size_t plan_bytes = L.plan_hdr + sizeof(uint32_t) * (size_t)n_items * n_kc;
+    L.plan_s = take(plan_bytes);
+    L.plan_t = take(plan_bytes);
+    L.bounds = take(sizeof(int4) * n_qblk);
+    L.cnt = take(sizeof(int) * n_items);
+    L.off = take(sizeof(int) * (n_items + 1));
     L.rows = take(sizeof(int32_t) * n_rows);
     L.qg = take((size_t)heads * n_rows * d * 2);
     L.od = take((size_t)heads * n_rows * d * 4);
@@ -145,7 +339,9 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows)
 
 size_t classify_workspace_bytes(const svga_problem *p, int n_rows)
 {
-    return classify_layout(p->heads, p->head_dim, n_rows).total;
+    return classify_layout(p->heads, p->head_dim, n_rows,
+                           p->num_frames * p->grid_h * p->grid_w)
+        .total;
 }
 
 svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
@@ -156,11 +352,15 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int H = p->heads, d = p->head_dim, S = p->grid_h * p->grid_w, N = p->num_frames * S;
-    const ClassifyLayout L = classify_layout(H, d, n_rows);
+    const ClassifyLayout L = classify_layout(H, d, n_rows, N);
     (void)ws_bytes;
     char *w = static_cast<char *>(ws);
-    int4 *info_s = reinterpret_cast<int4 *>(w + L.info_s);
-    int4 *info_t = reinterpret_cast<int4 *>(w + L.info_t);
+    char *plan_s = w + L.plan_s, *plan_t = w + L.plan_t;
+    int4 *info_s = reinterpret_cast<int4 *>(plan_s + sizeof(PlanHeader));
+    int4 *info_t = reinterpret_cast<int4 *>(plan_t + sizeof(PlanHeader));
+    int4 *bounds = reinterpret_cast<int4 *>(w + L.bounds);
+    int *cnt = reinterpret_cast<int *>(w + L.cnt);
+    int *off = reinterpret_cast<int *>(w + L.off);
     int32_t *rows_ws = reinterpret_cast<int32_t *>(w + L.rows);
     void *qg = w + L.qg;
     float *od = reinterpret_cast<float *>(w + L.od);
@@ -192,6 +392,19 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         gather_rows_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
                                                    static_cast<uint4 *>(qg), rows_use, N, n_rows,
                                                    status);
+    const int n_qblk = (n_rows + kBlockM - 1) / kBlockM, n_pairs = (n_qblk + 1) / 2;
+    const int n_items = H * n_pairs, n_kc = (N + 127) / 128;
+    row_bounds_kernel<<<n_qblk, 128, 0, st>>>(rows_use, n_rows, N, S, bounds);
+    for (char *plan : {plan_s, plan_t}) {
+        int4 *hinfo = reinterpret_cast<int4 *>(plan + sizeof(PlanHeader));
+        int4 *items = hinfo + H;
+        uint32_t *entries = reinterpret_cast<uint32_t *>(plan + L.plan_hdr);
+        pass_count_kernel<<<n_items, 256, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
+                                                   p->anchor_frame0, hinfo, bounds, cnt);
+        pass_items_kernel<<<1, 1024, 0, st>>>(H, n_pairs, n_items, N, n_kc, cnt, off, items, plan);
+        pass_write_kernel<<<n_items, 128, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
+                                                   p->anchor_frame0, hinfo, bounds, off, entries);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("classifier setup launch failed: %s", cudaGetErrorString(e));
@@ -213,19 +426,18 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.kn = 128;
     a.qrow_tokens = rows_use;
     a.out_f32 = 1;
-    const int n_qblk = (n_rows + kBlockM - 1) / kBlockM;
-    a.n_items = H * ((n_qblk + 1) / 2);
+    a.n_items = n_items;
     a.status = status;
     svga_status rc;
     a.mode = 1;
     a.head_info = nullptr;
     a.o = od;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
-    a.mode = 2;
-    a.head_info = reinterpret_cast<const int32_t *>(info_s);
+    a.mode = 0;  // the masked passes through their plans
+    a.plan = plan_s;
     a.o = os;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
-    a.head_info = reinterpret_cast<const int32_t *>(info_t);
+    a.plan = plan_t;
     a.o = ot;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
     double *partial = reinterpret_cast<double *>(w + L.partial);
