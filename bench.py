@@ -354,8 +354,13 @@ def run_svga(args, rank, world, local_rank):
                                                               scale, svga.FLAG_NAIVE_B1), reps)
     perm_ms = time_it(lambda: svga.svga_permute_tokens(qd, qp, prob), reps)
 
-    step_sep_ms = time_it(step_separate, reps)
-    step_ref_ms = time_it(step, reps)
+    # the two step forms timed alternately (order swapped each round): same clocks
+    sep_t, ref_t = [], []
+    for rnd in range(4):
+        for fn, acc in (((step_separate, sep_t), (step, ref_t)) if rnd % 2 == 0 else
+                        ((step, ref_t), (step_separate, sep_t))):
+            acc.append(time_it(fn, max(3, reps // 2)))
+    step_sep_ms, step_ref_ms = statistics.median(sep_t), statistics.median(ref_t)
     dense_flops = 4.0 * H * N * N * d
     # tile-aligned traversal (B3, opt-in): every pair of a visited tile is kept
     b3 = None

@@ -115,7 +115,8 @@ struct Item {
             if (naive) e &= ~(kEntF0 | kEntF1);
             return e;
         }
-        const bool full = (mode == 1) && !(ragged && n == n_kc - 1);
+        // dense: every chunk, full except a last one that runs past the final token
+        const bool full = !(ragged && n == n_kc - 1);
         uint32_t e = (uint32_t)n | kEntV0 | (full ? kEntF0 : 0u);
         if (valid1) e |= kEntV1 | (full ? kEntF1 : 0u);
         return e;
@@ -776,7 +777,7 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
             align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)a.heads + a.n_items), 256);
         kp.entries = reinterpret_cast<const uint32_t *>(plan + hdr);
     } else {
-        kp.head_info = reinterpret_cast<const int4 *>(a.head_info);
+        kp.head_info = nullptr;  // dense: no head info is read
         kp.items = nullptr;
         kp.entries = nullptr;
     }

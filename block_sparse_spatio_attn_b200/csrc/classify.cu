@@ -430,7 +430,6 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.status = status;
     svga_status rc;
     a.mode = 1;
-    a.head_info = nullptr;
     a.o = od;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
     a.mode = 0;  // the masked passes through their plans

@@ -77,7 +77,7 @@ struct AttnLaunch {
     int heads, nq_rows, nk_rows, d;
     int F, S, anchor;
     float scale;
-    int mode;                  // 0 plan, 1 dense (implicit), 2 masked everywhere (implicit)
+    int mode;                  // 0 plan, 1 dense (every chunk of every block pair)
     int naive;                 // plan mode: visit full tiles through the masked path
     int aligned;               // plan mode: keep every key of a visited tile (mask snapped to tiles)
     int part, num_parts;       // plan mode: run only the items of part `part` (0 of 1: all)
@@ -85,7 +85,6 @@ struct AttnLaunch {
     int qo_fm;                 // SVGA_FLAG_QO_FRAME_MAJOR: q, o, lse frame-major
     int kn;                    // keys per chunk: 64 or 128
     const void *plan;          // device plan (mode 0)
-    const int32_t *head_info;  // device int4 per head (modes 0 and 2)
     const int32_t *qrow_tokens;  // device [nq_rows] frame-major token of each query row (shared by all heads) or null
     int out_f32;               // o is float32 instead of bf16
     int n_items;
