@@ -63,7 +63,6 @@ __global__ void gather_rows_kernel(const uint4 *__restrict__ q, uint4 *__restric
 
 constexpr int kMseParts = 32;  // blocks per head in the first reduction stage
 
-// Stage 1: block (part, h) sums the squared deviations of one slice of head h.
 // Frame and in-frame index bounds (min f, max f, min s, max s) of each 128-row block of
 // sampled rows.  Rows outside 0..N-1 are clamped here (the gather reports them).
 __global__ void __launch_bounds__(128) row_bounds_kernel(const int32_t *rows, int n_rows, int N,
@@ -245,8 +244,63 @@ __global__ void __launch_bounds__(128) pass_write_kernel(int n_pairs, int n_qblk
     }
 }
 
+// The temporal pass takes the sampled rows grouped by in-frame index s (a counting sort
+// over the S positions), so that a 128-row block spans few positions and its plan skips
+// the key chunks out of band.  Each row's output does not depend on its block.
+__global__ void s_hist_kernel(const int32_t *rows, int n_rows, int N, int S, int *hist)
+{
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < n_rows; r += gridDim.x * blockDim.x) {
+        int t = __ldg(rows + r);
+        t = t < 0 ? 0 : (t >= N ? N - 1 : t);
+        atomicAdd(hist + t % S, 1);
+    }
+}
+
+// Exclusive scan of the S counts in place (one block).
+__global__ void __launch_bounds__(1024) s_scan_kernel(int *hist, int S)
+{
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int base = 0; base < S; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < S ? hist[i] : 0;
+        int x = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        int before = carry;
+        for (int j = 0; j < w; ++j) before += wsum[j];
+        if (i < S) hist[i] = before + x - v;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = before + x;
+        __syncthreads();
+    }
+}
+
+// rows_t[pos] = rows[r] with the rows of equal s contiguous; pos_t[r] = pos.
+__global__ void s_scatter_kernel(const int32_t *rows, int n_rows, int N, int S, int *cursor,
+                                 int32_t *rows_t, int32_t *pos_t)
+{
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < n_rows; r += gridDim.x * blockDim.x) {
+        const int t0 = __ldg(rows + r);
+        const int t = t0 < 0 ? 0 : (t0 >= N ? N - 1 : t0);
+        const int pos = atomicAdd(cursor + t % S, 1);
+        rows_t[pos] = t0;
+        pos_t[r] = pos;
+    }
+}
+
+// Stage 1: block (part, h) sums the squared deviations of one slice of head h.  ot holds
+// the temporal pass's rows in the grouped order: row r of od and os is row pos_t[r] there.
 __global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const float *os,
-                                                          const float *ot, int n, double *partial)
+                                                          const float *ot, const int32_t *pos_t,
+                                                          int d, int n, double *partial)
 {
     __shared__ double red[2][8];
     const int part = blockIdx.x, h = blockIdx.y;
@@ -255,8 +309,10 @@ __global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const
     const int i0 = part * per, i1 = min(n, i0 + per);
     double as = 0.0, at = 0.0;
     for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-        const double d = od[base + i];
-        const double a = os[base + i] - d, b = ot[base + i] - d;
+        const int r = i / d, c = i - r * d;
+        const double dv = od[base + i];
+        const double a = os[base + i] - dv;
+        const double b = ot[base + (size_t)__ldg(pos_t + r) * d + c] - dv;
         as += a * a;
         at += b * b;
     }
@@ -299,11 +355,11 @@ __global__ void mse_final_kernel(const double *partial, int heads, int n, int32_
 }
 
 struct ClassifyLayout {
-    size_t plan_s, plan_t, plan_hdr, bounds, cnt, off, rows, qg, od, os, ot, partial, types, mse,
-        status, total;
+    size_t plan_s, plan_t, plan_hdr, bounds, bounds_t, cnt, off, rows, rows_t, pos_t, s_hist, qg,
+        qg_t, od, os, ot, partial, types, mse, status, total;
 };
 
-ClassifyLayout classify_layout(int heads, int d, int n_rows, int N)
+ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
 {
     ClassifyLayout L{};
     size_t o = 0;
@@ -320,10 +376,15 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N)
     L.plan_s = take(plan_bytes);
     L.plan_t = take(plan_bytes);
     L.bounds = take(sizeof(int4) * n_qblk);
+    L.bounds_t = take(sizeof(int4) * n_qblk);
     L.cnt = take(sizeof(int) * n_items);
     L.off = take(sizeof(int) * (n_items + 1));
     L.rows = take(sizeof(int32_t) * n_rows);
+    L.rows_t = take(sizeof(int32_t) * n_rows);
+    L.pos_t = take(sizeof(int32_t) * n_rows);
+    L.s_hist = take(sizeof(int) * (size_t)S);
     L.qg = take((size_t)heads * n_rows * d * 2);
+    L.qg_t = take((size_t)heads * n_rows * d * 2);
     L.od = take((size_t)heads * n_rows * d * 4);
     L.os = take((size_t)heads * n_rows * d * 4);
     L.ot = take((size_t)heads * n_rows * d * 4);
@@ -340,7 +401,7 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N)
 size_t classify_workspace_bytes(const svga_problem *p, int n_rows)
 {
     return classify_layout(p->heads, p->head_dim, n_rows,
-                           p->num_frames * p->grid_h * p->grid_w)
+                           p->num_frames * p->grid_h * p->grid_w, p->grid_h * p->grid_w)
         .total;
 }
 
@@ -352,13 +413,18 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int H = p->heads, d = p->head_dim, S = p->grid_h * p->grid_w, N = p->num_frames * S;
-    const ClassifyLayout L = classify_layout(H, d, n_rows, N);
+    const ClassifyLayout L = classify_layout(H, d, n_rows, N, S);
     (void)ws_bytes;
     char *w = static_cast<char *>(ws);
     char *plan_s = w + L.plan_s, *plan_t = w + L.plan_t;
     int4 *info_s = reinterpret_cast<int4 *>(plan_s + sizeof(PlanHeader));
     int4 *info_t = reinterpret_cast<int4 *>(plan_t + sizeof(PlanHeader));
     int4 *bounds = reinterpret_cast<int4 *>(w + L.bounds);
+    int4 *bounds_t = reinterpret_cast<int4 *>(w + L.bounds_t);
+    int32_t *rows_t = reinterpret_cast<int32_t *>(w + L.rows_t);
+    int32_t *pos_t = reinterpret_cast<int32_t *>(w + L.pos_t);
+    int *s_hist = reinterpret_cast<int *>(w + L.s_hist);
+    void *qg_t = w + L.qg_t;
     int *cnt = reinterpret_cast<int *>(w + L.cnt);
     int *off = reinterpret_cast<int *>(w + L.off);
     int32_t *rows_ws = reinterpret_cast<int32_t *>(w + L.rows);
@@ -375,7 +441,8 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         bp.w_spatial[h] = (uint16_t)w_spatial[h];
         bp.w_temporal[h] = (uint16_t)w_temporal[h];
     }
-    if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) {
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess ||
+        cudaMemsetAsync(s_hist, 0, sizeof(int) * (size_t)S, st) != cudaSuccess) {
         set_error("cudaMemsetAsync failed");
         return SVGA_ERR_CUDA;
     }
@@ -394,16 +461,31 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
                                                    status);
     const int n_qblk = (n_rows + kBlockM - 1) / kBlockM, n_pairs = (n_qblk + 1) / 2;
     const int n_items = H * n_pairs, n_kc = (N + 127) / 128;
+    // rows grouped by in-frame index for the temporal pass, its Q rows gathered that way
+    const int sblocks = (n_rows + 255) / 256 < 1184 ? (n_rows + 255) / 256 : 1184;
+    s_hist_kernel<<<sblocks, 256, 0, st>>>(rows_use, n_rows, N, S, s_hist);
+    s_scan_kernel<<<1, 1024, 0, st>>>(s_hist, S);
+    s_scatter_kernel<<<sblocks, 256, 0, st>>>(rows_use, n_rows, N, S, s_hist, rows_t, pos_t);
+    if (vpr == 16)
+        gather_rows_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
+                                                    static_cast<uint4 *>(qg_t), rows_t, N, n_rows,
+                                                    status);
+    else
+        gather_rows_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
+                                                   static_cast<uint4 *>(qg_t), rows_t, N, n_rows,
+                                                   status);
     row_bounds_kernel<<<n_qblk, 128, 0, st>>>(rows_use, n_rows, N, S, bounds);
+    row_bounds_kernel<<<n_qblk, 128, 0, st>>>(rows_t, n_rows, N, S, bounds_t);
     for (char *plan : {plan_s, plan_t}) {
+        const int4 *bnd = plan == plan_s ? bounds : bounds_t;
         int4 *hinfo = reinterpret_cast<int4 *>(plan + sizeof(PlanHeader));
         int4 *items = hinfo + H;
         uint32_t *entries = reinterpret_cast<uint32_t *>(plan + L.plan_hdr);
         pass_count_kernel<<<n_items, 256, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
-                                                   p->anchor_frame0, hinfo, bounds, cnt);
+                                                   p->anchor_frame0, hinfo, bnd, cnt);
         pass_items_kernel<<<1, 1024, 0, st>>>(H, n_pairs, n_items, N, n_kc, cnt, off, items, plan);
         pass_write_kernel<<<n_items, 128, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
-                                                   p->anchor_frame0, hinfo, bounds, off, entries);
+                                                   p->anchor_frame0, hinfo, bnd, off, entries);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -437,10 +519,13 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.o = os;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
     a.plan = plan_t;
+    a.q = qg_t;
+    a.qrow_tokens = rows_t;
     a.o = ot;
     if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
     double *partial = reinterpret_cast<double *>(w + L.partial);
-    mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(od, os, ot, n_rows * d, partial);
+    mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(od, os, ot, pos_t, d, n_rows * d,
+                                                           partial);
     mse_final_kernel<<<(H + 127) / 128, 128, 0, st>>>(partial, H, n_rows * d, types, mse);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
