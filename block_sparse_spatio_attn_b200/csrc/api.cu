@@ -324,7 +324,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
         return SVGA_ERR_INVALID_ARG;
     }
     if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED | SVGA_FLAG_TEST_STALL |
-                  SVGA_FLAG_QO_FRAME_MAJOR)) {
+                  SVGA_FLAG_QO_FRAME_MAJOR | SVGA_FLAG_KV_FRAME_MAJOR)) {
         set_error("unknown flags 0x%x", flags);
         return SVGA_ERR_INVALID_ARG;
     }
@@ -363,6 +363,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     a.aligned = (flags & SVGA_FLAG_TILE_ALIGNED) ? 1 : 0;
     a.test_stall = (flags & SVGA_FLAG_TEST_STALL) ? 1 : 0;
     a.qo_fm = (flags & SVGA_FLAG_QO_FRAME_MAJOR) ? 1 : 0;
+    a.kv_fm = (flags & SVGA_FLAG_KV_FRAME_MAJOR) ? 1 : 0;
     a.kn = g.kn;
     a.plan = map->plan;
     a.n_items = g.n_items;

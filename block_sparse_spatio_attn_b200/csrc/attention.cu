@@ -57,6 +57,7 @@ constexpr uint32_t kNegInfBits = 0xff800000u;
 // warpgroups rise to kRegsHigh.  128 * kRegsLow + 256 * kRegsHigh must not exceed the
 // 384 * kRegsLaunch registers the CTA is launched with (checked on the host).
 constexpr int kRegsLaunch = 168, kRegsLow = 120, kRegsHigh = 192;
+constexpr int kGatherThreads = 64;  // warps 2 and 3, when K / V rows are gathered
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 struct KParams {
@@ -66,7 +67,8 @@ struct KParams {
     int n_items, part, num_parts;  // plan mode: this launch runs the items of one part
     int test_stall;                // test hook: the first K chunk is never loaded
     int qo_fm;                     // Q and O frame-major: Q rows gathered, O rows scattered
-    const void *q;                 // Q base (for the gather)
+    int kv_fm;                     // K and V frame-major: key rows gathered
+    const void *q, *k, *v;         // bases for the gathers
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -282,11 +284,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.mode == 0 && plan_item_of_block(p) >= p.n_items) return;  // the last group ran out
     const Item it = make_item(p, KN);
+    // keys of a head in a temporal-major order, read from frame-major K and V: warps 2
+    // and 3 gather the chunk rows instead of the TMA producer
+    const bool kv_gather = p.kv_fm && p.mode == 0 && __ldg(p.head_info + it.h).z != ORDER_FM;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bar->q_full), 1);  // the TMA load, or the last gathering warp
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(smem_u32(&bar->kv_full[s]), 1);
+            // the TMA load, or one arrival per gathering thread
+            mbar_init(smem_u32(&bar->kv_full[s]), kv_gather ? kGatherThreads : 1);
             mbar_init(smem_u32(&bar->kv_empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int issued = 0;
             bool ok = true;
-            for (int n = 0; n < it.E && ok; ++n) {
+            for (int n = 0; n < (kv_gather ? 0 : it.E) && ok; ++n) {
                 const int kc = (int)(it.entry(n) & kEntChunkMask);
                 for (int t = 0; t < 2; ++t) {
                     const int idx = 2 * n + t, s = idx % C::kStages, round = idx / C::kStages;
@@ -354,6 +360,79 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(p.test_stall && idx == 0))
                         mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
                                           (idx / C::kStages) & 1);
+            }
+        } else if (warp >= 2 && kv_gather) {
+            // ---------------------------------------------------- K/V row gather
+            // Chunk row r holds the key at position kc * KN + r of the head's order; its
+            // frame-major token is found by walking the order's grid.  Eight threads copy
+            // one 128-byte half row, 16 bytes each, into the 128-byte-swizzled stage (the
+            // layout the TMA load gives); rows past the last token are zero-filled.  A
+            // stage is handed over once its copies have landed and been made visible to
+            // the MMA (async proxy); one stage stays in flight behind the one issued.
+            const int gt = threadIdx.x - 64, u = gt & 7, r0 = gt >> 3;
+            const int korder = __ldg(p.head_info + it.h).z;
+            // within a head the row offsets fit 32 bits (at most 2^24 rows of 256 bytes)
+            const size_t head_off = (size_t)it.h * p.nk_rows * (D * 2);
+            const char *kb = static_cast<const char *>(p.k) + head_off;
+            const char *vb = static_cast<const char *>(p.v) + head_off;
+            const uint32_t dst_base = smem_u32(sKV) + r0 * 128 + ((u ^ r0) << 4);
+            const int total = 2 * it.E;
+            int tok[KN / 8];
+            bool ok = true;
+            for (int idx = 0; idx < total; ++idx) {
+                const int s = idx % C::kStages, round = idx / C::kStages;
+                if (round > 0 &&
+                    !mbar_wait(smem_u32(&bar->kv_empty[s]), (round - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (!(idx & 1)) {  // the K stage of a chunk: its rows' tokens
+                    const int pos0 = (int)(it.entry(idx >> 1) & kEntChunkMask) * KN + r0;
+                    int f = 0, sx = 0;
+                    if (pos0 < p.nk_rows) pos_to_coord(korder, pos0, p.F, p.S, f, sx);
+#pragma unroll
+                    for (int g = 0; g < KN / 8; ++g) {
+                        const int pos = pos0 + 8 * g;
+                        tok[g] = pos < p.nk_rows ? f * p.S + sx : -1;
+                        if (korder == ORDER_FM) {
+                            for (sx += 8; sx >= p.S; sx -= p.S) ++f;
+                        } else if (korder == ORDER_TM_STRICT) {
+                            for (f += 8; f >= p.F; f -= p.F) ++sx;
+                        } else if (f == 0) {  // the anchor frame leads the order
+                            sx += 8;
+                            if (sx >= p.S && pos + 8 < p.nk_rows)
+                                pos_to_coord(korder, pos + 8, p.F, p.S, f, sx);
+                        } else {
+                            for (f += 8; f >= p.F; f -= p.F - 1) ++sx;
+                        }
+                    }
+                }
+                if (!(p.test_stall && idx == 0)) {  // the test hook never loads stage 0
+                    const char *base = (idx & 1) ? vb : kb;
+                    const uint32_t dst = dst_base + s * C::kKVBytes;
+#pragma unroll
+                    for (int g = 0; g < KN / 8; ++g) {
+                        const char *src =
+                            base + ((uint32_t)(tok[g] < 0 ? 0 : tok[g]) * (D * 2) + u * 16);
+#pragma unroll
+                        for (int c = 0; c < D / 64; ++c)
+                            cp_async_16(dst + c * C::kKVChunk + g * 1024, src + c * 128,
+                                        tok[g] < 0 ? 0u : 16u);
+                    }
+                }
+                cp_async_commit();
+                if (idx > 0) {
+                    cp_async_wait_group<1>();  // stage idx - 1 has landed
+                    if (!(p.test_stall && idx == 1)) {
+                        fence_proxy_async_smem();
+                        mbar_arrive(smem_u32(&bar->kv_full[(idx - 1) % C::kStages]));
+                    }
+                }
+            }
+            cp_async_wait_group<0>();  // nothing in flight when the CTA exits
+            if (ok && total > 0) {
+                fence_proxy_async_smem();
+                mbar_arrive(smem_u32(&bar->kv_full[(total - 1) % C::kStages]));
             }
         } else if (warp == 1) {
             // --------------------------------------------------------- MMA issuer
@@ -764,7 +843,10 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.num_parts = a.num_parts > 0 ? a.num_parts : 1;
     kp.test_stall = a.test_stall;
     kp.qo_fm = a.qo_fm;
+    kp.kv_fm = a.kv_fm;
     kp.q = a.q;
+    kp.k = a.k;
+    kp.v = a.v;
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;

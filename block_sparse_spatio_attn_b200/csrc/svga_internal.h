@@ -83,6 +83,7 @@ struct AttnLaunch {
     int part, num_parts;       // plan mode: run only the items of part `part` (0 of 1: all)
     int test_stall;            // SVGA_FLAG_TEST_STALL: withhold the first K load
     int qo_fm;                 // SVGA_FLAG_QO_FRAME_MAJOR: q, o, lse frame-major
+    int kv_fm;                 // SVGA_FLAG_KV_FRAME_MAJOR: k, v frame-major
     int kn;                    // keys per chunk: 64 or 128
     const void *plan;          // device plan (mode 0)
     const int32_t *qrow_tokens;  // device [nq_rows] frame-major token of each query row (shared by all heads) or null

@@ -25,6 +25,7 @@ ORDER_FRAME_MAJOR, ORDER_TEMPORAL_MAJOR, ORDER_TEMPORAL_MAJOR_STRICT = 0, 1, 2
 FLAG_NAIVE_B1 = 1
 FLAG_TILE_ALIGNED = 2
 FLAG_QO_FRAME_MAJOR = 4
+FLAG_KV_FRAME_MAJOR = 8
 FLAG_TEST_STALL = 1 << 16
 
 EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",

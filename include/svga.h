@@ -93,6 +93,12 @@ enum {
      * ainews.tenesys.com, "Co sie zmienilo?" item 5; here only K and V move).
      * Results are identical bit for bit to permute -> attention -> unpermute. */
     SVGA_FLAG_QO_FRAME_MAJOR = 4,
+    /* k and v are FRAME-MAJOR for every head: the kernel reads the key rows of a head
+     * kept in a temporal-major order from their frame-major tokens (a gather of the
+     * chunk's rows into the same shared-memory layout the tile load gives), so the
+     * permutation of K and V is not needed either.  With SVGA_FLAG_QO_FRAME_MAJOR no
+     * tensor moves at all.  Results are identical bit for bit to the permuted call. */
+    SVGA_FLAG_KV_FRAME_MAJOR = 8,
     /* Test hook for the failure path: the first K chunk of every CTA is never loaded,
      * so the kernel's bounded waits run out (about one second per CTA wave), every role
      * stops, copies in flight are drained, TMEM is released and map->status reads
@@ -231,13 +237,15 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  * element (aihirek.info, section "A TPU-kernel kialakitasa ...").  An empty row
  * gives O = 0 and lse = -inf.
  *   q, k, v, o : DEVICE bf16 [heads, tokens, head_dim], every head in order[h]
- *                (q and o frame-major instead with SVGA_FLAG_QO_FRAME_MAJOR)
+ *                (q and o frame-major instead with SVGA_FLAG_QO_FRAME_MAJOR, k and v
+ *                with SVGA_FLAG_KV_FRAME_MAJOR)
  *   lse        : DEVICE float [heads, tokens] or NULL (frame-major with that flag)
  *   map        : built by svga_build_block_map (or _routed / _static) for this problem;
  *                the per-head type, band and order are read from the map's plan
  *   scale      : softmax scale, usually 1/sqrt(head_dim)
  *   flags      : 0 or a combination of SVGA_FLAG_NAIVE_B1 / SVGA_FLAG_TILE_ALIGNED
- *                (not both), SVGA_FLAG_QO_FRAME_MAJOR and the test hook
+ *                (not both), SVGA_FLAG_QO_FRAME_MAJOR, SVGA_FLAG_KV_FRAME_MAJOR and the
+ *                test hook
  *                SVGA_FLAG_TEST_STALL; other bits give SVGA_ERR_INVALID_ARG
  * bf16 inputs, fp32 accumulation and softmax, P rounded to bf16 for the PV product. */
 SVGA_API svga_status svga_sparse_attention_fwd(const void *q, const void *k, const void *v, void *o,

@@ -337,6 +337,65 @@ def test_qo_frame_major_equals_permuted_path(name, flags, tiles):
             assert_attn_close(on[h, rows], ro, ln[h, rows], rl, what=f"headline QO-FM head {h}")
 
 
+# ------------------------------- Q, K, V and O frame-major (nothing permuted)
+@pytest.mark.parametrize("name,flags,tiles,order", [
+    ("tiny", 0, None, C.ORDER_TEMPORAL_MAJOR), ("tiny", 0, (128, 64), C.ORDER_TEMPORAL_MAJOR_STRICT),
+    ("mid", 0, None, None), ("mid", svga.FLAG_NAIVE_B1, None, None),
+    ("mid", svga.FLAG_TILE_ALIGNED, (256, 128), None), ("mid", 0, (64, 64), None),
+    ("mid", 0, (128, 256), C.ORDER_TEMPORAL_MAJOR_STRICT), ("odd", 0, None, None),
+    ("headline", 0, None, None)])
+def test_all_frame_major_equals_permuted_path(name, flags, tiles, order):
+    """The kernel's gather of the key rows (K and V read from frame-major memory) fills
+    the stages with the same bits the tile load of permuted K and V gives: O and LSE
+    equal the permute -> attention -> unpermute path bit for bit, with K and V alone
+    frame-major and with every tensor frame-major."""
+    if name == "odd":   # one frame more than a power of two, rows not a multiple of 8
+        wl = C.Workload("odd_fm", 9, 5, 7, 64, [0, 1, 1], [1, 2, 0],
+                        [C.ORDER_FRAME_MAJOR, C.ORDER_TEMPORAL_MAJOR,
+                         C.ORDER_TEMPORAL_MAJOR_STRICT], seed=21)
+    else:
+        wl = C.ALL[name]()
+    if tiles:
+        wl = wl.with_tile(*tiles)
+    orders = wl.order if order is None else [order if t == C.TEMPORAL else o
+                                             for t, o in zip(wl.head_type, wl.order)]
+    q, k, v, qd, kd, vd = inputs(wl)
+    o_ref, lse_ref, _ = run_sparse_path(wl, qd, kd, vd, order=orders, flags=flags)
+    lse_fm = lse_to_frame_major(lse_ref.cpu().numpy(), wl, orders)
+    prob = svga.ProblemSpec.from_workload(wl, order=orders)
+    bmap = svga.build_block_map(prob)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    # K and V frame-major, Q and O in each head's order
+    qp = torch.empty_like(qd)
+    svga.svga_permute_tokens(qd, qp, prob)
+    op = torch.full_like(qd, float("nan"))
+    lse = torch.empty(wl.heads, wl.tokens, dtype=torch.float32, device="cuda")
+    svga.svga_sparse_attention_fwd(qp, kd, vd, op, lse, prob, bmap, scale,
+                                   flags | svga.FLAG_KV_FRAME_MAJOR)
+    o = torch.empty_like(qd)
+    svga.svga_unpermute_tokens(op, o, prob)
+    torch.cuda.synchronize()
+    assert bmap.device_status() == 0
+    assert torch.equal(o, o_ref)
+    assert torch.equal(lse, lse_ref)
+    # every tensor frame-major, in two parts
+    o = torch.full_like(qd, float("nan"))
+    for part in range(2):
+        svga.svga_sparse_attention_fwd_part(
+            qd, kd, vd, o, lse, prob, bmap, scale,
+            flags | svga.FLAG_QO_FRAME_MAJOR | svga.FLAG_KV_FRAME_MAJOR, part, 2)
+    torch.cuda.synchronize()
+    assert bmap.device_status() == 0
+    assert torch.equal(o, o_ref)
+    np.testing.assert_array_equal(lse.cpu().numpy(), lse_fm)
+    if name in ("odd", "headline") and flags == 0:
+        rows = sample_rows(wl, 96) if name == "headline" else np.arange(wl.tokens, dtype=np.int32)
+        on, ln = o.float().cpu().numpy(), lse.cpu().numpy()
+        for h in ((0, wl.heads - 1) if name == "headline" else range(wl.heads)):
+            ro, rl = oracle_rows(wl, q, k, v, h, rows)
+            assert_attn_close(on[h, rows], ro, ln[h, rows], rl, what=f"{name} all-FM head {h}")
+
+
 def test_maximum_head_count():
     """4,096 heads (the largest count the library takes), 2 frames of 4x6 tokens, d = 64:
     the per-head parameters travel as kernel parameters sized for that many heads.
