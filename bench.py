@@ -354,13 +354,17 @@ def run_svga(args, rank, world, local_rank):
                                                               scale, svga.FLAG_NAIVE_B1), reps)
     perm_ms = time_it(lambda: svga.svga_permute_tokens(qd, qp, prob), reps)
 
-    # the two step forms timed alternately (order swapped each round): same clocks
-    sep_t, ref_t = [], []
+    # the step forms timed alternately (order rotated each round): same clocks.  The
+    # all-frame-major form is one launch that also gathers the K and V rows itself.
+    def step_all_fm():
+        svga.svga_sparse_attention_fwd(qd, kd, vd, o, None, prob, bmap, scale,
+                                       svga.FLAG_QO_FRAME_MAJOR | svga.FLAG_KV_FRAME_MAJOR)
+
+    forms = [(step_separate, []), (step, []), (step_all_fm, [])]
     for rnd in range(4):
-        for fn, acc in (((step_separate, sep_t), (step, ref_t)) if rnd % 2 == 0 else
-                        ((step, ref_t), (step_separate, sep_t))):
+        for fn, acc in forms[rnd % 3:] + forms[:rnd % 3]:
             acc.append(time_it(fn, max(3, reps // 2)))
-    step_sep_ms, step_ref_ms = statistics.median(sep_t), statistics.median(ref_t)
+    step_sep_ms, step_ref_ms, step_fm_ms = (statistics.median(acc) for _, acc in forms)
     dense_flops = 4.0 * H * N * N * d
     # tile-aligned traversal (B3, opt-in): every pair of a visited tile is kept
     b3 = None
@@ -471,6 +475,9 @@ def run_svga(args, rank, world, local_rank):
         "sparse_over_dense": attn_ms / dense_ms, "target_ratio": kept_frac + 0.15,
         "naive_b1_ms": naive_ms, "tile_aligned_b3": b3,
         "step_with_separate_permutes": {"ms": step_sep_ms, "step_ms_same_conditions": step_ref_ms},
+        "step_all_frame_major": {"ms": step_fm_ms, "step_ms_same_conditions": step_ref_ms,
+                                 "launches": 1,
+                                 "note": "K and V rows gathered by the kernel (opt-in flag)"},
         "permute_ms_per_tensor": perm_ms, "map_build_ms": map_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
