@@ -108,19 +108,29 @@ def read_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def code_digest(src_path: str) -> str:
+    """sha256 of a C++/CUDA source with its // comments and blank lines removed, so that
+    an edit of the comments alone keeps the digest."""
+    lines = []
+    for line in open(src_path, encoding="utf-8"):
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def traffic_from_profile(kernel_src: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it
-    was taken on the current kernel source (sha256 recorded in the summary)."""
+    was taken on the current kernel code (code_sha256 recorded in the summary)."""
     path = os.path.join(ROOT, "profiles", "attention_headline_ncu.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
-    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_sha = re.search(r"code_sha256:\s*([0-9a-f]{64})", txt)
     m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt)
     if not (m_sha and m_b):
         return None
-    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
-    return float(m_b.group(1)) if sha == m_sha.group(1) else None
+    return float(m_b.group(1)) if code_digest(kernel_src) == m_sha.group(1) else None
 
 
 # ------------------------------------------------------------------ clock sampler

@@ -30,7 +30,10 @@
 //     chunk as full;
 //   * with Q and O frame-major, the softmax threads of a temporal-major head copy their
 //     own Q rows into the swizzled Q tile (frame-major heads keep the TMA load) and
-//     every head writes O and LSE rows back to their frame-major tokens.
+//     every head writes O and LSE rows back to their frame-major tokens;
+//   * with K and V frame-major, warps 2 and 3 gather the key chunks of a temporal-major
+//     head row by row (16-byte cp.async into the same swizzled stage layout) in place of
+//     warp 0's tile loads.
 //
 // Every mbarrier wait gives up after about a second: the CTA raises a shared abort
 // flag, drains its MMAs and copies, frees TMEM, writes SVGA_ERR_TIMEOUT to the
