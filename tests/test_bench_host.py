@@ -1,0 +1,29 @@
+"""Host logic of bench.py that needs no GPU: the digest that decides whether the
+committed ncu traffic figure still describes the kernel source."""
+
+
+def test_code_digest_ignores_comments_and_blank_lines(tmp_path):
+    import bench
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    c = tmp_path / "c.cu"
+    a.write_text("int f(int x)  // doubles\n{\n    return 2 * x;\n}\n")
+    b.write_text("// a new header comment\n\nint f(int x)\n{\n\n    return 2 * x;  // same\n}\n")
+    c.write_text("int f(int x)\n{\n    return 3 * x;\n}\n")
+    assert bench.code_digest(str(a)) == bench.code_digest(str(b))
+    assert bench.code_digest(str(a)) != bench.code_digest(str(c))
+
+
+def test_traffic_needs_a_matching_digest(tmp_path, monkeypatch):
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("__global__ void k() {}\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    summary = prof / "attention_headline_ncu.md"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    summary.write_text(f"code_sha256: {bench.code_digest(str(src))}\n"
+                       "dram_bytes_per_full_launch: 3.5e9\n")
+    assert bench.traffic_from_profile(str(src)) == 3.5e9
+    src.write_text("__global__ void k() { int x = 1; (void)x; }\n")
+    assert bench.traffic_from_profile(str(src)) is None
