@@ -111,3 +111,32 @@ def test_classify_size_validation(lib):
         svga.svga_classify_size(prob, 0)
     with pytest.raises(svga.SvgaError):
         svga.svga_classify_size(prob, 193)
+
+
+def test_sparse_forward_flag_and_part_checks_on_the_host(lib):
+    """Every flag combination is checked on the host before any CUDA call: unknown bits
+    and NAIVE with TILE_ALIGNED are rejected, TILE_ALIGNED needs tile_q >= 128, and the
+    accepted combinations (the frame-major ones included) get as far as the last host
+    check, the scale."""
+    P = ctypes.c_void_p
+    m = svga.BlockMapC()
+    m.plan, m.plan_bytes, m.status = 4096, 1 << 30, None   # never dereferenced here
+
+    def call(flags, scale=0.1, part=0, n=1, wl=C.mid()):
+        prob = svga.ProblemSpec.from_workload(wl)
+        return lib.svga_sparse_attention_fwd_part(
+            P(4096), P(4096), P(4096), P(4096), None, ctypes.byref(prob.c), ctypes.byref(m),
+            ctypes.c_float(scale), flags, part, n, P(0))
+
+    assert call(1 << 8) == 1 and b"unknown flags" in lib.svga_last_error()
+    assert call(svga.FLAG_NAIVE_B1 | svga.FLAG_TILE_ALIGNED) == 1
+    assert b"exclude" in lib.svga_last_error()
+    assert call(svga.FLAG_TILE_ALIGNED, wl=C.mid().with_tile(64, 64)) == 4
+    fm = svga.FLAG_QO_FRAME_MAJOR | svga.FLAG_KV_FRAME_MAJOR
+    for flags in (0, svga.FLAG_NAIVE_B1, svga.FLAG_TILE_ALIGNED, svga.FLAG_QO_FRAME_MAJOR,
+                  svga.FLAG_KV_FRAME_MAJOR, fm, fm | svga.FLAG_NAIVE_B1,
+                  fm | svga.FLAG_TILE_ALIGNED, fm | svga.FLAG_TEST_STALL):
+        assert call(flags, scale=-1.0) == 1, flags
+        assert b"scale" in lib.svga_last_error(), flags
+    assert call(0, part=2, n=2) == 1 and b"part" in lib.svga_last_error()
+    assert call(0, part=0, n=5000) == 1
