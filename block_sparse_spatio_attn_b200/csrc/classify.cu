@@ -283,7 +283,11 @@ __global__ void __launch_bounds__(1024) s_scan_kernel(int *hist, int S)
     }
 }
 
-// rows_t[pos] = rows[r] with the rows of equal s contiguous; pos_t[r] = pos.
+// rows_t[pos] = rows[r] with the rows of equal s contiguous; pos_t[r] = pos.  The order
+// among rows of one s follows the atomics and may change from call to call: a row's
+// output does not depend on the rows it shares a block with, the block's in-frame range
+// (all the temporal plan reads) does not change, and the deviation sums run in the
+// original row order, so the results are the same on every call.
 __global__ void s_scatter_kernel(const int32_t *rows, int n_rows, int N, int S, int *cursor,
                                  int32_t *rows_t, int32_t *pos_t)
 {
