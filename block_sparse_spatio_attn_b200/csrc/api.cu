@@ -1,6 +1,7 @@
 // api.cu -- the C entry points of svga.h: validation, sizes and launches.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -67,6 +68,21 @@ static svga_status validate_shape(const svga_problem *p, Geometry *g, int heads_
     if (!valid_tile(p->tile_q) || !valid_tile(p->tile_k)) {
         set_error("tile %dx%d unsupported (64, 128 or 256)", p->tile_q, p->tile_k);
         return SVGA_ERR_UNSUPPORTED;
+    }
+    {
+        // the CSR offsets and the plan's entry offsets are int32: the tile count (the
+        // lists' capacity) and the plan's entry capacity must fit
+        const long long tiles = (long long)p->heads * ((N + p->tile_q - 1) / p->tile_q) *
+                                ((N + p->tile_k - 1) / p->tile_k);
+        const long long kn = p->tile_k < 128 ? p->tile_k : 128;
+        const long long entries =
+            (long long)p->heads * (((N + kBlockM - 1) / kBlockM + 1) / 2) * ((N + kn - 1) / kn);
+        if (tiles > INT32_MAX || entries > INT32_MAX) {
+            set_error("problem too large: %lld tiles and %lld plan entries, int32 offsets "
+                      "hold at most %d",
+                      tiles, entries, INT32_MAX);
+            return SVGA_ERR_SHAPE;
+        }
     }
     const bool none_given = p->head_type == nullptr && p->band == nullptr && p->order == nullptr;
     if (heads_mode == kHeadsRequired || (heads_mode == kHeadsIfGiven && !none_given)) {

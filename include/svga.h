@@ -119,7 +119,10 @@ enum {
  *   order          per head: the token order Q, K, V (and O) of that head are in
  *   anchor_frame0  1: every query also keeps all keys of frame 0, the anchor
  *                  (aihirek.info, section "A Sparse VideoGen ..."); 0: no anchor
- *   tile_q, tile_k tile size of the block map: 64, 128 or 256 each */
+ *   tile_q, tile_k tile size of the block map: 64, 128 or 256 each
+ * Lists and plan are indexed with int32: heads * ceil(N/tile_q) * ceil(N/tile_k) and
+ * heads * ceil(N/256) * ceil(N/min(tile_k, 128)) must each stay below 2^31
+ * (SVGA_ERR_SHAPE otherwise). */
 typedef struct {
     int heads;
     int num_frames;

@@ -71,6 +71,12 @@ def _bad(lib, **kw):
     (dict(anchor_frame0=2), 1),
     (dict(num_frames=0), 2),
     (dict(grid_h=300, grid_w=300), 2),
+    # 64 heads x 1,105,425 tokens: 4.8e9 tiles overflow the int32 list offsets
+    (dict(heads=64, num_frames=17, grid_h=255, grid_w=255, head_type=[0] * 64,
+          band=[1] * 64, order=[0] * 64, tile_q=128, tile_k=128), 2),
+    # tile 256 in k: 1.1e9 tiles fit, but 2.4e9 plan entries (128-key chunks) do not
+    (dict(heads=64, num_frames=17, grid_h=255, grid_w=255, head_type=[0] * 64,
+          band=[1] * 64, order=[0] * 64, tile_q=256, tile_k=256), 2),
 ])
 def test_problem_validation(lib, kw, status):
     with pytest.raises(svga.SvgaError) as e:
