@@ -125,6 +125,45 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+class _Args:
+    """The tensor arguments of one call, checked for what the C ABI cannot see from a
+    pointer: the library reads and writes exactly the elements the problem implies, so
+    each tensor must have that dtype and shape (or element count) and be contiguous;
+    once all are checked, all must live on a CUDA device.  Raises SvgaError before
+    anything is launched."""
+
+    def __init__(self):
+        self.seen = []
+
+    def t(self, t, name: str, dtype, shape=None, numel=None, optional=False):
+        if t is None:
+            if optional:
+                return None
+            raise SvgaError(1, f"{name} is None")
+        if not isinstance(t, torch.Tensor):
+            raise SvgaError(1, f"{name} must be a torch.Tensor, got {type(t).__name__}")
+        if t.dtype != dtype:
+            raise SvgaError(1, f"{name} must be {dtype}, got {t.dtype}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise SvgaError(2, f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if numel is not None and t.numel() != numel:
+            raise SvgaError(2, f"{name} has {t.numel()} elements, expected {numel}")
+        if not t.is_contiguous():
+            raise SvgaError(1, f"{name} must be contiguous")
+        self.seen.append((name, t))
+        return _ptr(t)
+
+    def tokens(self, problem, **named):
+        """bf16 [heads, tokens, head_dim] tensors of a problem, in argument order."""
+        shape = (problem.heads, problem.tokens, problem.head_dim)
+        return [self.t(t, n, torch.bfloat16, shape) for n, t in named.items()]
+
+    def done(self):
+        for name, t in self.seen:
+            if not t.is_cuda:
+                raise SvgaError(1, f"{name} must be on a CUDA device")
+
+
 @dataclass
 class ProblemSpec:
     """A problem with its host arrays kept alive for the C struct."""
@@ -218,21 +257,29 @@ def svga_validate_block_map(problem: ProblemSpec, bmap: BlockMap, stream=None) -
 
 def svga_permute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                         stream=None) -> torch.Tensor:
-    _check(load().svga_permute_tokens(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
-                                      _stream(stream)))
+    a = _Args()
+    ps, pd = a.tokens(problem, src=src, dst=dst)
+    a.done()
+    _check(load().svga_permute_tokens(ps, pd, ctypes.byref(problem.c), _stream(stream)))
     return dst
 
 
 def svga_unpermute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                           stream=None) -> torch.Tensor:
-    _check(load().svga_unpermute_tokens(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
-                                        _stream(stream)))
+    a = _Args()
+    ps, pd = a.tokens(problem, src=src, dst=dst)
+    a.done()
+    _check(load().svga_unpermute_tokens(ps, pd, ctypes.byref(problem.c), _stream(stream)))
     return dst
 
 
 def svga_sparse_attention_fwd(q, k, v, o, lse, problem: ProblemSpec, bmap: BlockMap,
                               scale: float, flags: int = 0, stream=None) -> torch.Tensor:
-    _check(load().svga_sparse_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+    a = _Args()
+    pq, pk, pv, po = a.tokens(problem, q=q, k=k, v=v, o=o)
+    pl = a.t(lse, "lse", torch.float32, (problem.heads, problem.tokens), optional=True)
+    a.done()
+    _check(load().svga_sparse_attention_fwd(pq, pk, pv, po, pl,
                                             ctypes.byref(problem.c), ctypes.byref(bmap.c),
                                             float(scale), int(flags), _stream(stream)))
     return o
@@ -241,18 +288,28 @@ def svga_sparse_attention_fwd(q, k, v, o, lse, problem: ProblemSpec, bmap: Block
 def svga_sparse_attention_fwd_part(q, k, v, o, lse, problem: ProblemSpec, bmap: BlockMap,
                                    scale: float, flags: int, part: int, num_parts: int,
                                    stream=None) -> torch.Tensor:
+    a = _Args()
+    pq, pk, pv, po = a.tokens(problem, q=q, k=k, v=v, o=o)
+    pl = a.t(lse, "lse", torch.float32, (problem.heads, problem.tokens), optional=True)
+    a.done()
     _check(load().svga_sparse_attention_fwd_part(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(problem.c),
-        ctypes.byref(bmap.c), float(scale), int(flags), int(part), int(num_parts),
-        _stream(stream)))
+        pq, pk, pv, po, pl, ctypes.byref(problem.c), ctypes.byref(bmap.c),
+        float(scale), int(flags), int(part), int(num_parts), _stream(stream)))
     return o
 
 
 def svga_dense_attention_fwd(q, k, v, o, lse, scale: float, status=None,
                              stream=None) -> torch.Tensor:
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise SvgaError(2, "q must be a [heads, tokens, head_dim] tensor")
     H, N, d = q.shape
-    _check(load().svga_dense_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                           H, N, d, float(scale), _ptr(status),
+    a = _Args()
+    pq, pk, pv, po = (a.t(t, n, torch.bfloat16, (H, N, d))
+                      for n, t in (("q", q), ("k", k), ("v", v), ("o", o)))
+    pl = a.t(lse, "lse", torch.float32, (H, N), optional=True)
+    pst = a.t(status, "status", torch.int32, numel=1, optional=True)
+    a.done()
+    _check(load().svga_dense_attention_fwd(pq, pk, pv, po, pl, H, N, d, float(scale), pst,
                                            _stream(stream)))
     return o
 
@@ -267,15 +324,21 @@ def svga_classify_heads(q, k, v, problem: ProblemSpec, w_spatial, w_temporal, ro
                         scale: float, workspace: Optional[torch.Tensor] = None, stream=None):
     """Returns (head_type list, mse [heads, 2] list).  Synchronises the stream."""
     H = problem.heads
+    a = _Args()
+    pq, pk, pv = a.tokens(problem, q=q, k=k, v=v)
+    pr = a.t(rows, "rows", torch.int32, numel=int(n_rows), optional=True)
+    a.done()
     ws_bytes = svga_classify_size(problem, n_rows)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    a.t(workspace, "workspace", torch.uint8)
+    a.done()
     types = (ctypes.c_int32 * H)()
     mse = (ctypes.c_float * (2 * H))()
     wsp = (ctypes.c_int32 * H)(*w_spatial)
     wtp = (ctypes.c_int32 * H)(*w_temporal)
-    _check(load().svga_classify_heads(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(problem.c),
-                                      wsp, wtp, _ptr(rows), int(n_rows), float(scale),
+    _check(load().svga_classify_heads(pq, pk, pv, ctypes.byref(problem.c),
+                                      wsp, wtp, pr, int(n_rows), float(scale),
                                       types, mse, _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
     return list(types), [[mse[2 * h], mse[2 * h + 1]] for h in range(H)]
@@ -288,23 +351,34 @@ def svga_classify_heads_async(q, k, v, problem: ProblemSpec, w_spatial, w_tempor
                               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Head types (and deviations, status) written to device tensors; no synchronisation."""
     H = problem.heads
+    a = _Args()
+    pq, pk, pv = a.tokens(problem, q=q, k=k, v=v)
+    pr = a.t(rows, "rows", torch.int32, numel=int(n_rows), optional=True)
+    pt = a.t(head_type_dev, "head_type_dev", torch.int32, numel=H)
+    pm = a.t(mse_dev, "mse_dev", torch.float32, numel=2 * H, optional=True)
+    ps = a.t(status_dev, "status_dev", torch.int32, numel=1, optional=True)
+    a.done()
     if workspace is None:
         workspace = torch.empty(svga_classify_size(problem, n_rows), dtype=torch.uint8,
                                 device=q.device)
+    a.t(workspace, "workspace", torch.uint8)
+    a.done()
     wsp = (ctypes.c_int32 * H)(*w_spatial)
     wtp = (ctypes.c_int32 * H)(*w_temporal)
     _check(load().svga_classify_heads_async(
-        _ptr(q), _ptr(k), _ptr(v), ctypes.byref(problem.c), wsp, wtp, _ptr(rows), int(n_rows),
-        float(scale), _ptr(head_type_dev), _ptr(mse_dev), _ptr(status_dev), _ptr(workspace),
-        workspace.numel(), _stream(stream)))
+        pq, pk, pv, ctypes.byref(problem.c), wsp, wtp, pr, int(n_rows), float(scale), pt, pm,
+        ps, _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def svga_build_block_map_routed(problem: ProblemSpec, head_type_dev: torch.Tensor, w_spatial,
                                 w_temporal, bmap: BlockMap, stream=None) -> BlockMap:
     H = problem.heads
+    a = _Args()
+    pt = a.t(head_type_dev, "head_type_dev", torch.int32, numel=H)
+    a.done()
     wsp = (ctypes.c_int32 * H)(*w_spatial)
     wtp = (ctypes.c_int32 * H)(*w_temporal)
-    _check(load().svga_build_block_map_routed(ctypes.byref(problem.c), _ptr(head_type_dev), wsp,
+    _check(load().svga_build_block_map_routed(ctypes.byref(problem.c), pt, wsp,
                                               wtp, ctypes.byref(bmap.c), _ptr(bmap.workspace),
                                               bmap.workspace.numel(), _stream(stream)))
     return bmap
@@ -312,14 +386,20 @@ def svga_build_block_map_routed(problem: ProblemSpec, head_type_dev: torch.Tenso
 
 def svga_permute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                                bmap: BlockMap, stream=None) -> torch.Tensor:
-    _check(load().svga_permute_tokens_mapped(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
+    a = _Args()
+    ps, pd = a.tokens(problem, src=src, dst=dst)
+    a.done()
+    _check(load().svga_permute_tokens_mapped(ps, pd, ctypes.byref(problem.c),
                                              ctypes.byref(bmap.c), _stream(stream)))
     return dst
 
 
 def svga_unpermute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                                  bmap: BlockMap, stream=None) -> torch.Tensor:
-    _check(load().svga_unpermute_tokens_mapped(_ptr(src), _ptr(dst), ctypes.byref(problem.c),
+    a = _Args()
+    ps, pd = a.tokens(problem, src=src, dst=dst)
+    a.done()
+    _check(load().svga_unpermute_tokens_mapped(ps, pd, ctypes.byref(problem.c),
                                                ctypes.byref(bmap.c), _stream(stream)))
     return dst
 
