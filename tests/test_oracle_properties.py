@@ -1,0 +1,70 @@
+"""Randomised pins of the oracle's mask, kept count, tile counts, tile classes and CSR
+lists (CPU only).  For small random problems (frames, grid, head type, band, anchor, token
+order, tile sizes with ragged tails), everything on the reference side is recomputed here
+by brute force: the mask from its definition with numpy broadcasting, the token orders
+from their position formulas, tile counts by summing the reordered, zero-padded mask,
+classes and lists from the counts.  The reference side calls nothing in the oracle."""
+import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle
+
+
+def tokens_of_positions(order, F, S):
+    """Frame-major token at each position of `order`, from the orders' definitions:
+    frame-major t = f*S + s; strict temporal-major position s*F + f; anchor-first:
+    frame 0 at positions 0..S-1, then frame f >= 1 at S + s*(F-1) + (f-1)."""
+    tok = np.empty(F * S, np.int64)
+    for f in range(F):
+        for s in range(S):
+            if order == oracle.FRAME_MAJOR:
+                p = f * S + s
+            elif order == oracle.TEMPORAL_STRICT:
+                p = s * F + f
+            else:
+                p = s if f == 0 else S + s * (F - 1) + (f - 1)
+            tok[p] = f * S + s
+    return tok
+
+
+def brute_mask(type_, band, anchor, F, S):
+    t = np.arange(F * S)
+    f, s = t // S, t % S
+    if type_ == oracle.SPATIAL:
+        near = np.abs(f[:, None] - f[None, :]) <= band
+    else:
+        near = np.abs(s[:, None] - s[None, :]) <= band
+    return near | (bool(anchor) & (f[None, :] == 0))
+
+
+@settings(max_examples=150, deadline=None)
+@given(F=st.integers(1, 6), gh=st.integers(1, 6), gw=st.integers(1, 8),
+       type_=st.sampled_from([oracle.SPATIAL, oracle.TEMPORAL]), band=st.integers(0, 9),
+       anchor=st.integers(0, 1),
+       order=st.sampled_from([oracle.FRAME_MAJOR, oracle.TEMPORAL_ANCHOR_FIRST,
+                              oracle.TEMPORAL_STRICT]),
+       tq=st.sampled_from([8, 16, 24, 32, 48, 64]), tk=st.sampled_from([8, 16, 20, 32, 64]))
+def test_oracle_tiles_match_brute_force(F, gh, gw, type_, band, anchor, order, tq, tk):
+    S = gh * gw
+    N = F * S
+    m = brute_mask(type_, band, anchor, F, S)
+    assert oracle.kept_count(type_, band, anchor, F, S) == int(m.sum())
+    np.testing.assert_array_equal(oracle.mask(type_, band, anchor, F, S), m.astype(np.uint8))
+
+    tok = tokens_of_positions(order, F, S)
+    mp = m[np.ix_(tok, tok)]                       # the mask in position order
+    nq, nk = -(-N // tq), -(-N // tk)
+    pad = np.zeros((nq * tq, nk * tk), np.int64)
+    pad[:N, :N] = mp
+    counts = pad.reshape(nq, tq, nk, tk).sum(axis=(1, 3))
+    cls = np.where(counts == 0, 0, np.where(counts == tq * tk, 1, 2)).astype(np.uint8)
+
+    got = oracle.tile_map(type_, band, anchor, order, F, S, tq, tk)
+    np.testing.assert_array_equal(got["counts"], counts)
+    np.testing.assert_array_equal(got["cls"], cls)
+    for c, ptr, idx in ((1, "full_ptr", "full_idx"), (2, "bnd_ptr", "bnd_idx")):
+        rows = [np.nonzero(cls[i] == c)[0] for i in range(nq)]
+        np.testing.assert_array_equal(got[ptr], np.cumsum([0] + [len(r) for r in rows]))
+        np.testing.assert_array_equal(got[idx], np.concatenate(rows).astype(np.int32)
+                                      if rows else np.zeros(0, np.int32))
