@@ -68,3 +68,32 @@ def test_oracle_tiles_match_brute_force(F, gh, gw, type_, band, anchor, order, t
         np.testing.assert_array_equal(got[ptr], np.cumsum([0] + [len(r) for r in rows]))
         np.testing.assert_array_equal(got[idx], np.concatenate(rows).astype(np.int32)
                                       if rows else np.zeros(0, np.int32))
+
+
+@settings(max_examples=60, deadline=None)
+@given(F=st.integers(1, 5), gh=st.integers(1, 5), gw=st.integers(1, 6),
+       d=st.sampled_from([4, 8, 16]),
+       type_=st.sampled_from([oracle.SPATIAL, oracle.TEMPORAL]), band=st.integers(0, 6),
+       anchor=st.integers(0, 1), seed=st.integers(0, 2 ** 16),
+       scale=st.floats(0.05, 2.0))
+def test_oracle_attention_matches_library_sdpa(F, gh, gw, d, type_, band, anchor, seed,
+                                               scale):
+    """O against torch's fp64 scaled_dot_product_attention under the brute-force mask, LSE
+    against torch.logsumexp; rows with no kept key (possible without the anchor only if
+    the band excludes the query itself, which it never does) are not produced here."""
+    import torch
+    S = gh * gw
+    N = F * S
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn(N, d, generator=g, dtype=torch.float64).float() for _ in range(3))
+    m = torch.from_numpy(brute_mask(type_, band, anchor, F, S))
+    rows = np.arange(N, dtype=np.int32)
+    o, lse = oracle.attention_rows(q.numpy(), k.numpy(), v.numpy(), F, S, scale, type_, band,
+                                   anchor, rows)
+    qd, kd, vd = q.double(), k.double(), v.double()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qd[None], kd[None], vd[None], attn_mask=m[None], scale=scale)[0]
+    logits = (qd @ kd.T) * scale
+    ref_lse = torch.logsumexp(logits.masked_fill(~m, float("-inf")), dim=1)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
