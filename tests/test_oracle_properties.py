@@ -97,3 +97,44 @@ def test_oracle_attention_matches_library_sdpa(F, gh, gw, d, type_, band, anchor
     ref_lse = torch.logsumexp(logits.masked_fill(~m, float("-inf")), dim=1)
     np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
+
+
+@settings(max_examples=60, deadline=None)
+@given(F=st.integers(1, 5), gh=st.integers(1, 5), gw=st.integers(1, 6),
+       type_=st.sampled_from([oracle.SPATIAL, oracle.TEMPORAL]), band=st.integers(0, 6),
+       anchor=st.integers(0, 1),
+       order=st.sampled_from([oracle.FRAME_MAJOR, oracle.TEMPORAL_ANCHOR_FIRST,
+                              oracle.TEMPORAL_STRICT]),
+       tq=st.sampled_from([4, 8, 12, 16]), tk=st.sampled_from([4, 8, 10, 16]),
+       seed=st.integers(0, 2 ** 16))
+def test_oracle_tile_aligned_matches_library_sdpa(F, gh, gw, type_, band, anchor, order, tq,
+                                                  tk, seed):
+    """The tile-aligned traversal keeps every key of each (q-tile, k-tile) of the head's
+    token order that holds an exactly kept pair.  That snapped mask is built here from
+    brute-force tile counts and mapped back to frame-major tokens; the oracle gets the
+    same counts and must match torch's fp64 SDPA under it."""
+    import torch
+    S = gh * gw
+    N = F * S
+    d, scale = 8, 0.3
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn(N, d, generator=g, dtype=torch.float64).float() for _ in range(3))
+    tok = tokens_of_positions(order, F, S)
+    mp = brute_mask(type_, band, anchor, F, S)[np.ix_(tok, tok)]
+    nq, nk = -(-N // tq), -(-N // tk)
+    pad = np.zeros((nq * tq, nk * tk), np.int64)
+    pad[:N, :N] = mp
+    counts = pad.reshape(nq, tq, nk, tk).sum(axis=(1, 3))
+    snapped_pos = (counts[np.arange(N)[:, None] // tq, np.arange(N)[None, :] // tk] > 0)
+    snapped = np.zeros((N, N), bool)
+    snapped[np.ix_(tok, tok)] = snapped_pos          # back to frame-major tokens
+    rows = np.arange(N, dtype=np.int32)
+    o, lse = oracle.attention_rows_tile_aligned(q.numpy(), k.numpy(), v.numpy(), F, S, scale,
+                                                order, tq, tk, counts, 0, rows)
+    m = torch.from_numpy(snapped)
+    qd, kd, vd = q.double(), k.double(), v.double()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qd[None], kd[None], vd[None], attn_mask=m[None], scale=scale)[0]
+    ref_lse = torch.logsumexp(((qd @ kd.T) * scale).masked_fill(~m, float("-inf")), dim=1)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
