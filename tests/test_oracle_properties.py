@@ -138,3 +138,36 @@ def test_oracle_tile_aligned_matches_library_sdpa(F, gh, gw, type_, band, anchor
     ref_lse = torch.logsumexp(((qd @ kd.T) * scale).masked_fill(~m, float("-inf")), dim=1)
     np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
+
+
+@settings(max_examples=40, deadline=None)
+@given(F=st.integers(2, 5), gh=st.integers(1, 5), gw=st.integers(2, 6),
+       w_s=st.integers(0, 3), w_t=st.integers(0, 8), anchor=st.integers(0, 1),
+       n_rows=st.integers(1, 12), seed=st.integers(0, 2 ** 16))
+def test_oracle_classifier_matches_library_sdpa(F, gh, gw, w_s, w_t, anchor, n_rows, seed):
+    """Deviations of the spatial and temporal outputs from the dense one (mean square over
+    the sampled rows x d) and the choice (the smaller, a tie to spatial), with the three
+    outputs from torch's fp64 SDPA under the brute-force masks."""
+    import torch
+    S = gh * gw
+    N = F * S
+    d, scale = 8, 0.4
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn(N, d, generator=g, dtype=torch.float64).float() for _ in range(3))
+    rows = np.sort(np.random.default_rng(seed).choice(N, size=min(n_rows, N),
+                                                      replace=False)).astype(np.int32)
+    qd, kd, vd = q.double(), k.double(), v.double()
+
+    def sdpa(mask):
+        m = torch.from_numpy(mask)
+        return torch.nn.functional.scaled_dot_product_attention(
+            qd[None], kd[None], vd[None], attn_mask=m[None], scale=scale)[0].numpy()[rows]
+
+    od = sdpa(np.ones((N, N), bool))
+    ms = float(np.mean((sdpa(brute_mask(oracle.SPATIAL, w_s, anchor, F, S)) - od) ** 2))
+    mt = float(np.mean((sdpa(brute_mask(oracle.TEMPORAL, w_t, anchor, F, S)) - od) ** 2))
+    t, ms_o, mt_o = oracle.classify(q.numpy(), k.numpy(), v.numpy(), F, S, scale, w_s, w_t,
+                                    anchor, rows)
+    assert abs(ms_o - ms) <= 1e-12 and abs(mt_o - mt) <= 1e-12
+    if abs(ms - mt) > 1e-12:
+        assert t == (oracle.SPATIAL if ms < mt else oracle.TEMPORAL)
