@@ -171,3 +171,15 @@ def test_oracle_classifier_matches_library_sdpa(F, gh, gw, w_s, w_t, anchor, n_r
     assert abs(ms_o - ms) <= 1e-12 and abs(mt_o - mt) <= 1e-12
     if abs(ms - mt) > 1e-12:
         assert t == (oracle.SPATIAL if ms < mt else oracle.TEMPORAL)
+
+
+@settings(max_examples=80, deadline=None)
+@given(F=st.integers(1, 9), S=st.integers(1, 40),
+       order=st.sampled_from([oracle.FRAME_MAJOR, oracle.TEMPORAL_ANCHOR_FIRST,
+                              oracle.TEMPORAL_STRICT]))
+def test_oracle_permutation_matches_the_order_formulas(F, S, order):
+    """oracle.permutation (position -> frame-major token) equals the order written out
+    from its position formula, and is a permutation of 0..N-1."""
+    perm = oracle.permutation(order, F, S)
+    np.testing.assert_array_equal(perm, tokens_of_positions(order, F, S))
+    np.testing.assert_array_equal(np.sort(perm), np.arange(F * S))
