@@ -27,3 +27,26 @@ def test_traffic_needs_a_matching_digest(tmp_path, monkeypatch):
     assert bench.traffic_from_profile(str(src)) == 3.5e9
     src.write_text("__global__ void k() { int x = 1; (void)x; }\n")
     assert bench.traffic_from_profile(str(src)) is None
+
+
+def test_flop_accounting_matches_the_mask_on_random_problems():
+    """bench.py's kept-pair and per-row kept-key counts (closed forms, the metric's FLOP)
+    against the mask written out with numpy, on random small problems."""
+    import numpy as np
+
+    import bench
+    from block_sparse_spatio_attn_b200 import configs as C
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        F, S = int(rng.integers(1, 8)), int(rng.integers(1, 30))
+        t = int(rng.integers(0, 2))
+        w, a = int(rng.integers(0, 10)), int(rng.integers(0, 2))
+        tok = np.arange(F * S)
+        f, s = tok // S, tok % S
+        near = (np.abs(f[:, None] - f[None, :]) if t == C.SPATIAL
+                else np.abs(s[:, None] - s[None, :])) <= w
+        m = near | (bool(a) & (f[None, :] == 0))
+        assert bench.kept_pairs(t, w, a, F, S) == int(m.sum())
+        wl = C.Workload("r", F, 1, S, 64, [t], [w], [0], seed=0, anchor_frame0=a)
+        for r in rng.choice(F * S, size=min(5, F * S), replace=False):
+            assert bench.kept_keys_of_row(wl, 0, int(r)) == int(m[r].sum())
