@@ -50,3 +50,28 @@ def test_flop_accounting_matches_the_mask_on_random_problems():
         wl = C.Workload("r", F, 1, S, 64, [t], [w], [0], seed=0, anchor_frame0=a)
         for r in rng.choice(F * S, size=min(5, F * S), replace=False):
             assert bench.kept_keys_of_row(wl, 0, int(r)) == int(m[r].sum())
+
+
+def test_reference_arm_rank_contract():
+    """bench.py --impl reference: rank 0 prints one JSON line with the oracle's figures,
+    any other rank exits 0 without work or output (the torchrun launch)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config",
+           "tiny", "--steps", "1", "--warmup", "3", "--ref-step-seconds", "0.2"]
+    outs = {}
+    for rank in (0, 1):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1")
+        r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=300, cwd=root)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs[rank] = [l for l in r.stdout.splitlines() if l.strip()]
+    assert outs[1] == []
+    assert len(outs[0]) == 1
+    line = json.loads(outs[0][0])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["n_gpus"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["gpu_launches"] == 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
