@@ -146,3 +146,44 @@ def test_sparse_forward_flag_and_part_checks_on_the_host(lib):
         assert b"scale" in lib.svga_last_error(), flags
     assert call(0, part=2, n=2) == 1 and b"part" in lib.svga_last_error()
     assert call(0, part=0, n=5000) == 1
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "svga.h"
+int main(void)
+{
+    int type[2] = {SVGA_HEAD_SPATIAL, SVGA_HEAD_TEMPORAL}, band[2] = {1, 8};
+    int order[2] = {SVGA_ORDER_FRAME_MAJOR, SVGA_ORDER_TEMPORAL_MAJOR};
+    svga_problem p = {2, 3, 8, 8, 64, type, band, order, 1, 64, 64};
+    size_t cls = 0, ptr = 0, plan = 0, ws = 0;
+    int64_t fcap = 0, bcap = 0;
+    svga_status rc = svga_block_map_size(&p, &cls, &ptr, &fcap, &bcap, &plan, &ws);
+    p.head_dim = 96;
+    svga_status bad = svga_block_map_size(&p, &cls, &ptr, &fcap, &bcap, &plan, &ws);
+    printf("%d %d %zu %zu %lld %s %s\n", svga_version(), (int)rc, cls, ptr, (long long)fcap,
+           svga_status_string(bad), svga_last_error());
+    return rc == SVGA_OK && bad == SVGA_ERR_UNSUPPORTED ? 0 : 1;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    """A C99 program includes include/svga.h (pedantic, no warnings), links libsvga.so
+    and calls host-side entry points: the ABI needs no C++ and no Python."""
+    import subprocess
+    src = tmp_path / "use_svga.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_svga"
+    libdir = os.path.join(ROOT, "block_sparse_spatio_attn_b200")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lsvga", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    ver, rc, cls, ptr, fcap, bad = r.stdout.split()[:6]
+    assert int(ver) == lib.svga_version() and int(rc) == 0
+    assert (int(cls), int(ptr), int(fcap)) == (2 * 3 * 3, 4 * (2 * 3 + 1), 2 * 3 * 3)
+    assert bad == "SVGA_ERR_UNSUPPORTED" and "head_dim 96" in r.stdout
