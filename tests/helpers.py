@@ -100,15 +100,38 @@ def assert_attn_close(o_gpu: np.ndarray, o_ref: np.ndarray, lse_gpu=None, lse_re
     return max_abs, rel
 
 
-def sample_rows(wl, per_head: int = 160, seed: int = 0) -> np.ndarray:
-    """Deterministic row sample: a few whole 128-row blocks (first, middle, the ragged
-    last one) plus spread rows."""
+def kernel_blocks(N: int) -> list:
+    """Indices of the 128-row query blocks a row sample covers whole: the first work item
+    (blocks 0 and 1: one block per softmax warpgroup), a middle pair (an even and the odd
+    block after it), and the last two blocks (the ragged last block and its neighbour)."""
+    nb = -(-N // 128)
+    mid = (nb // 2) // 2 * 2
+    return sorted({b for b in (0, 1, mid, mid + 1, nb - 2, nb - 1) if 0 <= b < nb})
+
+
+def block_rows(wl, orders=None) -> np.ndarray:
+    """Frame-major tokens of every row of kernel_blocks(N), for each token order in
+    `orders` (default: the orders of the workload's heads).  A query block is a run of
+    128 consecutive positions of the head's order, so for a temporal-major head its rows
+    are scattered over the frame-major tokens."""
+    N, F, S = wl.tokens, wl.frames, wl.tokens_per_frame
+    orders = sorted(set(wl.order if orders is None else orders))
+    rows = set()
+    for od in orders:
+        perm = oracle.permutation(od, F, S)   # position -> frame-major token
+        for b in kernel_blocks(N):
+            rows.update(perm[b * 128: min(N, b * 128 + 128)].tolist())
+    return np.array(sorted(rows), np.int32)
+
+
+def sample_rows(wl, per_head: int = 160, seed: int = 0, orders=None) -> np.ndarray:
+    """Deterministic row sample (frame-major tokens): every row of the whole 128-row
+    query blocks of kernel_blocks(N) in each head's token order (block_rows: all 128 TMEM
+    lanes of both softmax warpgroups, and the ragged last block), the last 16 tokens,
+    plus `per_head` spread rows."""
     N = wl.tokens
     rng = np.random.default_rng(seed)
-    blocks = [0, (N // 128) // 2 * 128, (N - 1) // 128 * 128]
-    rows = set()
-    for b in blocks:
-        rows.update(range(b, min(N, b + 32)))
+    rows = set(block_rows(wl, orders).tolist())
     rows.update(range(max(0, N - 16), N))
-    rows.update(rng.choice(N, size=max(0, per_head - len(rows)), replace=False).tolist())
+    rows.update(rng.choice(N, size=min(N, per_head), replace=False).tolist())
     return np.array(sorted(rows), np.int32)

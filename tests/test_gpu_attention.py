@@ -2,7 +2,9 @@
 
 Tolerance (bf16 inputs, fp32 accumulation): max-abs 2e-2, relative Frobenius 1e-2,
 LSE max-abs 1e-3.  Full-size workloads are checked on sampled rows, including whole
-128-row blocks and the ragged last block."""
+128-row query blocks in each head's token order (first, middle and last work items,
+both blocks of each, so every TMEM lane of both softmax warpgroups) and the ragged last
+block."""
 import math
 
 import numpy as np
@@ -84,7 +86,8 @@ def test_mid_tile_sizes(tq, tk):
 
 def test_mid_frame_major_temporal():
     wl = C.mid()
-    check_sparse(wl, rows=sample_rows(wl, 200, seed=3), order=[C.ORDER_FRAME_MAJOR] * 4)
+    check_sparse(wl, rows=sample_rows(wl, 200, seed=3, orders=[C.ORDER_FRAME_MAJOR]),
+                 order=[C.ORDER_FRAME_MAJOR] * 4)
 
 
 def test_headline_sparse_sampled():
@@ -198,7 +201,8 @@ def test_mid_tile_aligned_frame_major_temporal():
     """Temporal heads left frame-major: most visited tiles are boundary tiles there, so
     snapping keeps many more pairs than the exact mask."""
     wl = C.mid()
-    check_tile_aligned(wl, rows=sample_rows(wl, 200), order=[C.ORDER_FRAME_MAJOR] * wl.heads)
+    check_tile_aligned(wl, rows=sample_rows(wl, 200, orders=[C.ORDER_FRAME_MAJOR]),
+                       order=[C.ORDER_FRAME_MAJOR] * wl.heads)
 
 
 def test_headline_tile_aligned():
