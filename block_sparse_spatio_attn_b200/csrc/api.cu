@@ -139,6 +139,11 @@ size_t plan_header_bytes(const Geometry &g)
 
 int64_t plan_entry_cap(const Geometry &g) { return (int64_t)g.n_items * g.n_kc; }
 
+size_t plan_bytes_needed(const Geometry &g)
+{
+    return plan_header_bytes(g) + sizeof(uint32_t) * (size_t)plan_entry_cap(g);
+}
+
 static svga_status check_tensor(const void *p, const char *name)
 {
     if (!p) {
@@ -162,6 +167,69 @@ static svga_status check_launch(const char *what)
     return SVGA_OK;
 }
 
+svga_status check_map_outputs(const Geometry &g, const svga_block_map *map)
+{
+    if (!map || !map->cls || !map->full_ptr || !map->full_idx || !map->bnd_ptr || !map->bnd_idx ||
+        !map->plan) {
+        set_error("block map buffers must be non-NULL device pointers");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!aligned(map->plan, 256) || !aligned(map->full_ptr, 4) || !aligned(map->bnd_ptr, 4) ||
+        !aligned(map->full_idx, 4) || !aligned(map->bnd_idx, 4)) {
+        set_error("plan must be 256-byte aligned, CSR arrays 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    // The plan's worst case is required: a build into a smaller plan would have to drop
+    // entries while its items still count them.
+    if (map->plan_bytes < plan_bytes_needed(g) || map->full_cap < 0 || map->bnd_cap < 0) {
+        set_error("plan (%zu bytes, needs %zu) smaller than svga_block_map_size, or a negative "
+                  "list capacity",
+                  map->plan_bytes, plan_bytes_needed(g));
+        return SVGA_ERR_WORKSPACE;
+    }
+    return SVGA_OK;
+}
+
+svga_status check_map_plan(const Geometry &g, const svga_block_map *map)
+{
+    if (!map || !map->plan) {
+        set_error("block map or its plan is NULL");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!aligned(map->plan, 256)) {
+        set_error("the block map's plan must be 256-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (map->plan_bytes < plan_bytes_needed(g)) {
+        set_error("block map plan (%zu bytes) smaller than svga_block_map_size (%zu) for this "
+                  "problem",
+                  map->plan_bytes, plan_bytes_needed(g));
+        return SVGA_ERR_INVALID_ARG;
+    }
+    return SVGA_OK;
+}
+
+static svga_status check_map_buffers(const Geometry &g, const svga_block_map *map,
+                                     const void *workspace, size_t workspace_bytes)
+{
+    svga_status rc = check_map_outputs(g, map);
+    if (rc != SVGA_OK) return rc;
+    if (!workspace) {
+        set_error("the build workspace must be a non-NULL device pointer");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!aligned(workspace, 256)) {
+        set_error("the build workspace must be 256-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (workspace_bytes < block_map_workspace_bytes(g)) {
+        set_error("workspace (%zu < %zu) smaller than svga_block_map_size", workspace_bytes,
+                  block_map_workspace_bytes(g));
+        return SVGA_ERR_WORKSPACE;
+    }
+    return SVGA_OK;
+}
+
 }  // namespace svga
 
 using namespace svga;
@@ -180,30 +248,8 @@ svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes, 
     if (ptr_bytes) *ptr_bytes = sizeof(int32_t) * ((size_t)g.heads * g.n_q + 1);
     if (full_cap) *full_cap = tiles;
     if (bnd_cap) *bnd_cap = tiles;
-    if (plan_bytes) *plan_bytes = plan_header_bytes(g) + sizeof(uint32_t) * (size_t)plan_entry_cap(g);
+    if (plan_bytes) *plan_bytes = plan_bytes_needed(g);
     if (workspace_bytes) *workspace_bytes = block_map_workspace_bytes(g);
-    return SVGA_OK;
-}
-
-static svga_status check_map_buffers(const Geometry &g, const svga_block_map *map,
-                                     const void *workspace, size_t workspace_bytes)
-{
-    if (!map || !map->cls || !map->full_ptr || !map->full_idx || !map->bnd_ptr || !map->bnd_idx ||
-        !map->plan || !workspace) {
-        set_error("block map buffers and workspace must be non-NULL device pointers");
-        return SVGA_ERR_INVALID_ARG;
-    }
-    if (!aligned(map->plan, 256) || !aligned(workspace, 256) || !aligned(map->full_ptr, 4) ||
-        !aligned(map->bnd_ptr, 4) || !aligned(map->full_idx, 4) || !aligned(map->bnd_idx, 4)) {
-        set_error("plan and workspace must be 256-byte aligned, CSR arrays 4-byte aligned");
-        return SVGA_ERR_ALIGNMENT;
-    }
-    if (workspace_bytes < block_map_workspace_bytes(g) || map->plan_bytes < plan_header_bytes(g) ||
-        map->full_cap < 0 || map->bnd_cap < 0) {
-        set_error("workspace (%zu < %zu) or plan (%zu) smaller than svga_block_map_size",
-                  workspace_bytes, block_map_workspace_bytes(g), map->plan_bytes);
-        return SVGA_ERR_WORKSPACE;
-    }
     return SVGA_OK;
 }
 
@@ -273,10 +319,7 @@ static svga_status permute_mapped_common(const void *src, void *dst, const svga_
     Geometry g;
     svga_status rc = validate_shape(problem, &g, kHeadsSkip);
     if (rc != SVGA_OK) return rc;
-    if (!map || !map->plan || map->plan_bytes < plan_header_bytes(g)) {
-        set_error("block map plan missing or smaller than svga_block_map_size");
-        return SVGA_ERR_INVALID_ARG;
-    }
+    if ((rc = check_map_plan(g, map)) != SVGA_OK) return rc;
     if ((rc = check_tensor(src, "src")) != SVGA_OK || (rc = check_tensor(dst, "dst")) != SVGA_OK)
         return rc;
     const size_t bytes = (size_t)g.heads * g.N * g.d * 2;
@@ -285,8 +328,7 @@ static svga_status permute_mapped_common(const void *src, void *dst, const svga_
         set_error("src and dst overlap");
         return SVGA_ERR_INVALID_ARG;
     }
-    return launch_permute(src, dst, problem, g, inverse, stream,
-                          static_cast<const char *>(map->plan) + sizeof(PlanHeader));
+    return launch_permute(src, dst, problem, g, inverse, stream, map->plan, map->status);
 }
 
 svga_status svga_permute_tokens_mapped(const void *src, void *dst, const svga_problem *problem,
@@ -335,10 +377,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
         set_error("lse is not 4-byte aligned");
         return SVGA_ERR_ALIGNMENT;
     }
-    if (!map || !map->plan || map->plan_bytes < plan_header_bytes(g)) {
-        set_error("block map plan missing or smaller than svga_block_map_size");
-        return SVGA_ERR_INVALID_ARG;
-    }
+    if ((rc = check_map_plan(g, map)) != SVGA_OK) return rc;
     if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED | SVGA_FLAG_TEST_STALL |
                   SVGA_FLAG_QO_FRAME_MAJOR | SVGA_FLAG_KV_FRAME_MAJOR)) {
         set_error("unknown flags 0x%x", flags);
@@ -381,6 +420,9 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     a.qo_fm = (flags & SVGA_FLAG_QO_FRAME_MAJOR) ? 1 : 0;
     a.kv_fm = (flags & SVGA_FLAG_KV_FRAME_MAJOR) ? 1 : 0;
     a.kn = g.kn;
+    a.tile_q = g.tile_q;
+    a.tile_k = g.tile_k;
+    a.check_plan = 1;  // the map is the caller's: its header must describe this problem
     a.plan = map->plan;
     a.n_items = g.n_items;
     a.part = part;

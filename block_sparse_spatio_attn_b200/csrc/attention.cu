@@ -72,6 +72,9 @@ struct KParams {
     int qo_fm;                     // Q and O frame-major: Q rows gathered, O rows scattered
     int kv_fm;                     // K and V frame-major: key rows gathered
     const void *q, *k, *v;         // bases for the gathers
+    int check_plan;                // compare the plan with this launch before using it
+    int tile_q, tile_k;            // the map tiles the plan must have been built with
+    const PlanHeader *hdr;
     const int4 *items;
     const uint32_t *entries;
     const int4 *head_info;
@@ -135,6 +138,30 @@ __device__ __forceinline__ int plan_item_of_block(const KParams &p)
 {
     const int g = blockIdx.x, r = p.part, n = p.num_parts;
     return g * n + ((g & 1) ? n - 1 - r : r);
+}
+
+// A caller's plan must describe this launch before any of its offsets is used: the
+// header against the launch's shape, tiles, anchor and item count, then this CTA's work
+// item (head, even first block, entry range inside the plan) and the head's info.
+// Every thread of the CTA reads the same words, so the verdict is uniform.
+__device__ __forceinline__ bool plan_matches(const KParams &p, int kn)
+{
+    const int4 *h4 = reinterpret_cast<const int4 *>(p.hdr);
+    // {magic, heads, tokens, frames}, {tokens_per_frame, anchor, tile_q, tile_k},
+    // {kn, n_qblk, n_kc, n_items}, {entry_cap (low, high), reserved}
+    const int4 a = __ldg(h4), b = __ldg(h4 + 1), c = __ldg(h4 + 2), d = __ldg(h4 + 3);
+    const long long entry_cap = (long long)(uint32_t)d.x | ((long long)d.y << 32);
+    if (!(a.x == kPlanMagic && a.y == p.heads && a.z == p.nq_rows && a.z == p.nk_rows &&
+          a.w == p.F && b.x == p.S && b.y == p.anchor && b.z == p.tile_q && b.w == p.tile_k &&
+          c.x == kn && c.y == p.n_qblk && c.z == p.n_kc && c.w == p.n_items))
+        return false;
+    const int4 x = __ldg(p.items + plan_item_of_block(p));
+    if (!(x.x >= 0 && x.x < p.heads && x.y >= 0 && !(x.y & 1) && x.y < p.n_qblk && x.z >= 0 &&
+          x.w >= 0 && x.w <= p.n_kc && (long long)x.z + x.w <= entry_cap))
+        return false;
+    const int4 hi = __ldg(p.head_info + x.x);
+    return (hi.x == MASK_SPATIAL || hi.x == MASK_TEMPORAL) && hi.y >= 0 && hi.z >= ORDER_FM &&
+           hi.z <= ORDER_TM_STRICT;
 }
 
 __device__ __forceinline__ Item make_item(const KParams &p, int kn)
@@ -286,6 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.mode == 0 && plan_item_of_block(p) >= p.n_items) return;  // the last group ran out
+    if (p.mode == 0 && p.check_plan && !plan_matches(p, KN)) {
+        // a map built for another problem: report it and touch nothing
+        if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int32_t)SVGA_ERR_INVALID_ARG);
+        return;
+    }
     const Item it = make_item(p, KN);
     // keys of a head in a temporal-major order, read from frame-major K and V: warps 2
     // and 3 gather the chunk rows instead of the TMA producer
@@ -853,8 +885,12 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.n_qblk = (a.nq_rows + kBlockM - 1) / kBlockM;
     kp.n_pairs = (kp.n_qblk + 1) / 2;
     kp.n_kc = (a.nk_rows + a.kn - 1) / a.kn;
+    kp.check_plan = a.check_plan;
+    kp.tile_q = a.tile_q;
+    kp.tile_k = a.tile_k;
     if (a.mode == 0) {
         const char *plan = static_cast<const char *>(a.plan);
+        kp.hdr = reinterpret_cast<const PlanHeader *>(plan);
         kp.head_info = reinterpret_cast<const int4 *>(plan + sizeof(PlanHeader));
         kp.items = kp.head_info + a.heads;
         // entries start after header + head_info + items, 256-byte aligned
@@ -862,6 +898,7 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
             align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)a.heads + a.n_items), 256);
         kp.entries = reinterpret_cast<const uint32_t *>(plan + hdr);
     } else {
+        kp.hdr = nullptr;
         kp.head_info = nullptr;  // dense: no head info is read
         kp.items = nullptr;
         kp.entries = nullptr;

@@ -10,16 +10,20 @@
 // kStaticScratchBytes, which every GPU that loads the library holds until the process
 // exits.
 //
-// The array is a host-side stand-in in host code: its device address is looked up once
-// per device (cudaGetSymbolAddress, with that device current) on the first call made on
-// that device, and cached.  That first call should therefore happen before any stream
-// capture.  All calls share the one array and it keeps the previous call's contents;
-// the build writes every scratch word it reads before reading it, so nothing needs
-// clearing, but two calls that overlap on the GPU (different streams, no ordering
-// between them) race on the array.
+// In host code the name g_map_scratch does not denote device memory: it is a host-side
+// stand-in for the array, and a kernel given it would fault or read the wrong memory.
+// The device address is therefore asked for with cudaGetSymbolAddress on every call, in
+// the CUDA context current at that call (one host call, no allocation, no
+// synchronisation).  Looking it up each time keeps the address right after a
+// cudaDeviceReset or when another context of the device is current.  The first call in
+// a context may load the library's device code into it, so make that first call before
+// any stream capture.
+//
+// All calls share the one array and it keeps the previous call's contents; the build
+// writes every scratch word it reads before reading it, so nothing needs clearing, but
+// two calls that overlap on the GPU (different streams, no ordering between them) race
+// on the array.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "svga_internal.h"
 
@@ -31,32 +35,16 @@ static_assert(kStaticScratchBytes == SVGA_MAP_STATIC_SCRATCH_BYTES, "header and 
 
 __device__ __align__(256) unsigned char g_map_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_map_scratch on the current device (looked up once per device).
+// Device address of g_map_scratch in the current context.
 svga_status scratch_address(void **out)
 {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        set_error("cudaGetDevice failed or device ordinal out of range: %s",
-                  cudaGetErrorString(e));
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_map_scratch);
+    if (e != cudaSuccess || !p) {
+        set_error("cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
         return SVGA_ERR_CUDA;
     }
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_map_scratch);
-        if (e != cudaSuccess || !p) {
-            set_error("cudaGetSymbolAddress of the static scratch failed: %s",
-                      cudaGetErrorString(e));
-            return SVGA_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return SVGA_OK;
 }
 
@@ -71,11 +59,6 @@ extern "C" svga_status svga_build_block_map_static(const svga_problem *problem,
     Geometry g;
     svga_status rc = validate_problem(problem, &g);
     if (rc != SVGA_OK) return rc;
-    if (!map || !map->cls || !map->full_ptr || !map->full_idx || !map->bnd_ptr || !map->bnd_idx ||
-        !map->plan) {
-        set_error("block map buffers must be non-NULL device pointers");
-        return SVGA_ERR_INVALID_ARG;
-    }
     const size_t need = block_map_workspace_bytes(g);
     if (need > kStaticScratchBytes) {
         set_error("this problem needs %zu bytes of build scratch, more than the %zu bytes of the "
@@ -83,18 +66,7 @@ extern "C" svga_status svga_build_block_map_static(const svga_problem *problem,
                   need, kStaticScratchBytes);
         return SVGA_ERR_WORKSPACE;
     }
-    auto misaligned = [](const void *p, uintptr_t a) {
-        return (reinterpret_cast<uintptr_t>(p) % a) != 0;
-    };
-    if (misaligned(map->plan, 256) || misaligned(map->full_ptr, 4) || misaligned(map->bnd_ptr, 4) ||
-        misaligned(map->full_idx, 4) || misaligned(map->bnd_idx, 4)) {
-        set_error("plan must be 256-byte aligned, CSR arrays 4-byte aligned");
-        return SVGA_ERR_ALIGNMENT;
-    }
-    if (map->plan_bytes < plan_header_bytes(g) || map->full_cap < 0 || map->bnd_cap < 0) {
-        set_error("plan (%zu bytes) smaller than svga_block_map_size", map->plan_bytes);
-        return SVGA_ERR_WORKSPACE;
-    }
+    if ((rc = check_map_outputs(g, map)) != SVGA_OK) return rc;
     void *scratch = nullptr;
     if ((rc = scratch_address(&scratch)) != SVGA_OK) return rc;
     return launch_build_block_map(problem, g, map, scratch, kStaticScratchBytes, stream);

@@ -19,14 +19,29 @@ struct OrderParams {
     uint8_t order[kMaxHeads];
 };
 
+// Does a block map's plan (header, then head info) describe this launch?  Checked by
+// every block before anything is written, so a map of another problem changes nothing.
+__device__ __forceinline__ bool plan_fits(const int4 *plan, int heads, int N, int F, int S, int h)
+{
+    const int4 a = __ldg(plan), b = __ldg(plan + 1);  // {magic, heads, tokens, frames}, {S, ..}
+    if (!(a.x == kPlanMagic && a.y == heads && a.z == N && a.w == F && b.x == S)) return false;
+    const int order = __ldg(plan + 4 + h).z;  // head info follows the 64-byte header
+    return order >= ORDER_FM && order <= ORDER_TM_STRICT;
+}
+
 template <int VPR>  // 16-byte vectors per row (head_dim / 8)
 __global__ void __launch_bounds__(256) permute_kernel(const uint4 *__restrict__ src,
                                                       uint4 *__restrict__ dst, int N, int F, int S,
                                                       int inverse, OrderParams op,
-                                                      const int4 *__restrict__ head_info)
+                                                      const int4 *__restrict__ plan,
+                                                      int32_t *status)
 {
     const int h = blockIdx.y;
-    const int order = head_info ? head_info[h].z : op.order[h];
+    if (plan && !plan_fits(plan, gridDim.y, N, F, S, h)) {
+        if (threadIdx.x == 0 && status) atomicCAS(status, 0, (int32_t)SVGA_ERR_INVALID_ARG);
+        return;
+    }
+    const int order = plan ? __ldg(plan + 4 + h).z : op.order[h];
     const size_t head_off = (size_t)h * N * VPR;
     const int total = N * VPR;
     for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
@@ -49,11 +64,12 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4 *__restrict__ 
 }  // namespace
 
 svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
-                           int inverse, void *stream, const void *plan_head_info)
+                           int inverse, void *stream, const void *plan, int32_t *status)
 {
+    static_assert(sizeof(PlanHeader) == 4 * sizeof(int4), "head info starts at int4 index 4");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     OrderParams op;
-    const int4 *hi = static_cast<const int4 *>(plan_head_info);
+    const int4 *hi = static_cast<const int4 *>(plan);
     for (int h = 0; h < g.heads; ++h) op.order[h] = hi ? 0 : (uint8_t)p->order[h];
     const int vpr = g.d / 8;
     const int total = g.N * vpr;
@@ -63,11 +79,11 @@ svga_status launch_permute(const void *src, void *dst, const svga_problem *p, co
     if (vpr == 16)
         permute_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
                                                  static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op,
-                                                 hi);
+                                                 hi, status);
     else
         permute_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(src),
                                                 static_cast<uint4 *>(dst), g.N, g.F, g.S, inverse, op,
-                                                hi);
+                                                hi, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("permute launch failed: %s", cudaGetErrorString(e));

@@ -14,8 +14,8 @@ enum { MASK_SPATIAL = 0, MASK_TEMPORAL = 1, MASK_DENSE = 2 };
 
 constexpr int kMaxHeads = 4096;
 constexpr int kMaxTokens = 1 << 24;
-constexpr int kBlockM = 128;
-constexpr int kMaxParts = 4096;  // largest num_parts of a partitioned attention call  // query rows per tcgen05 tile (one TMEM lane per row)
+constexpr int kBlockM = 128;     // query rows per tcgen05 tile (one TMEM lane per row)
+constexpr int kMaxParts = 4096;  // largest num_parts of a partitioned attention call
 
 // Execution plan of the attention kernel, stored in svga_block_map::plan.
 //   PlanHeader, then int4 head_info[heads] = {mask type, band, order, 0},
@@ -51,7 +51,15 @@ svga_status validate_problem(const svga_problem *p, Geometry *g);
 svga_status validate_geometry(const svga_problem *p, Geometry *g);
 size_t plan_header_bytes(const Geometry &g);  // header + head_info + items, 256-aligned
 int64_t plan_entry_cap(const Geometry &g);
+// Plan bytes a map of this geometry needs (header + worst-case entries): what
+// svga_block_map_size reports and every call that takes a map requires.
+size_t plan_bytes_needed(const Geometry &g);
 size_t align_up(size_t x, size_t a);
+// Output buffers of a map build (everything but the workspace): non-NULL, aligned, and a
+// plan of at least plan_bytes_needed.  Shared by the workspace and the static builds.
+svga_status check_map_outputs(const Geometry &g, const svga_block_map *map);
+// The plan of a map handed to a call that reads it (attention, mapped permutations).
+svga_status check_map_plan(const Geometry &g, const svga_block_map *map);
 
 // block_map.cu
 // Per-head type, band and order come from the problem's host arrays, or, when types_dev
@@ -66,8 +74,11 @@ size_t block_map_workspace_bytes(const Geometry &g);
 
 // permute.cu
 // Per-head order from the problem's host array, or from a plan's head info when set.
+// With a plan, its header is checked against the geometry on the device first: on a
+// mismatch nothing is written and `status` (when not NULL) is set to SVGA_ERR_INVALID_ARG.
 svga_status launch_permute(const void *src, void *dst, const svga_problem *p, const Geometry &g,
-                           int inverse, void *stream, const void *plan_head_info = nullptr);
+                           int inverse, void *stream, const void *plan = nullptr,
+                           int32_t *status = nullptr);
 
 // attention.cu
 struct AttnLaunch {
@@ -85,6 +96,8 @@ struct AttnLaunch {
     int qo_fm;                 // SVGA_FLAG_QO_FRAME_MAJOR: q, o, lse frame-major
     int kv_fm;                 // SVGA_FLAG_KV_FRAME_MAJOR: k, v frame-major
     int kn;                    // keys per chunk: 64 or 128
+    int tile_q, tile_k;        // plan mode: the problem's map tiles
+    int check_plan;            // plan mode: compare the plan's header and items with the call
     const void *plan;          // device plan (mode 0)
     const int32_t *qrow_tokens;  // device [nq_rows] frame-major token of each query row (shared by all heads) or null
     int out_f32;               // o is float32 instead of bf16

@@ -61,7 +61,7 @@ extern "C" svga_status svga_validate_block_map(const svga_problem *problem,
     svga_status rc = validate_geometry(problem, &g);
     if (rc != SVGA_OK) return rc;
     if (!map || !map->cls || !map->full_ptr || !map->bnd_ptr || !map->plan ||
-        map->plan_bytes < plan_header_bytes(g)) {
+        map->plan_bytes < plan_bytes_needed(g)) {
         set_error("block map buffers missing or plan smaller than svga_block_map_size");
         return SVGA_ERR_INVALID_ARG;
     }
@@ -130,7 +130,8 @@ extern "C" svga_status svga_validate_block_map(const svga_problem *problem,
     PlanHeader hdr;
     std::memcpy(&hdr, head.data(), sizeof hdr);
     if (hdr.magic != kPlanMagic || hdr.heads != g.heads || hdr.tokens != g.N ||
-        hdr.frames != g.F || hdr.tokens_per_frame != g.S || hdr.tile_q != g.tile_q ||
+        hdr.frames != g.F || hdr.tokens_per_frame != g.S ||
+        hdr.anchor != problem->anchor_frame0 || hdr.tile_q != g.tile_q ||
         hdr.tile_k != g.tile_k || hdr.kn != g.kn || hdr.n_qblk != g.n_qblk ||
         hdr.n_kc != g.n_kc || hdr.n_items != g.n_items)
         return fail("plan header does not match the problem", hdr.magic, hdr.n_items);

@@ -151,6 +151,9 @@ typedef struct {
  *             internal to the library
  *   status    int32 device word or NULL; cleared by each call that takes the map,
  *             set to an svga_status by a kernel that fails on the device.
+ * Every call that builds or reads a map requires plan_bytes to be at least
+ * svga_block_map_size's plan_bytes for the call's problem (the worst case, so a build
+ * never drops entries); a smaller plan is rejected on the host.
  * Full/boundary specialisation: full tiles take an unmasked fast path, only
  * boundary tiles are masked by coordinates (aihirek.info, section "A TPU-kernel
  * kialakitasa ..."; ainews.tenesys.com, "Co sie zmienilo?" item 2). */
@@ -198,8 +201,11 @@ SVGA_API svga_status svga_build_block_map(const svga_problem *problem, svga_bloc
  *     SVGA_MAP_STATIC_SCRATCH_BYTES that each GPU loading the library keeps until the
  *     process exits.  A problem needing more scratch (svga_block_map_size's
  *     workspace_bytes) is rejected with SVGA_ERR_WORKSPACE and nothing is launched.
- *   - The first call on a device looks up the array's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the CUDA context current at
+ *     that call (cudaGetSymbolAddress: no allocation, no synchronisation), so the call
+ *     stays correct after a cudaDeviceReset or with another context of the device
+ *     current.  The first call in a context may load the library's device code into
+ *     it: make that first call before any stream capture.
  *   - The call allocates nothing.  All calls share the array: calls that overlap on the
  *     GPU (unordered streams) race; calls ordered on one stream are safe.
  * Results are identical to svga_build_block_map's. */
@@ -244,7 +250,11 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  *                with SVGA_FLAG_KV_FRAME_MAJOR)
  *   lse        : DEVICE float [heads, tokens] or NULL (frame-major with that flag)
  *   map        : built by svga_build_block_map (or _routed / _static) for this problem;
- *                the per-head type, band and order are read from the map's plan
+ *                the per-head type, band and order are read from the map's plan.  The
+ *                kernel first compares the plan's header (magic, heads, tokens, frames,
+ *                grid, anchor, tiles, chunk size and item count) and each work item
+ *                with this call: a map built for another problem sets map->status to
+ *                SVGA_ERR_INVALID_ARG and nothing is written (O and lse untouched)
  *   scale      : softmax scale, usually 1/sqrt(head_dim)
  *   flags      : 0 or a combination of SVGA_FLAG_NAIVE_B1 / SVGA_FLAG_TILE_ALIGNED
  *                (not both), SVGA_FLAG_QO_FRAME_MAJOR, SVGA_FLAG_KV_FRAME_MAJOR and the
@@ -349,7 +359,10 @@ SVGA_API svga_status svga_build_block_map_routed(const svga_problem *problem,
                                         svga_stream_t stream);
 
 /* svga_permute_tokens / svga_unpermute_tokens with each head's order read from the
- * plan of `map` on the device instead of problem->order. */
+ * plan of `map` on the device instead of problem->order.  The plan's header and head
+ * info are checked against the problem on the device first: a map built for another
+ * problem sets map->status (when not NULL) to SVGA_ERR_INVALID_ARG and dst is left
+ * untouched.  The status word is not cleared by these calls. */
 SVGA_API svga_status svga_permute_tokens_mapped(const void *src, void *dst,
                                        const svga_problem *problem, const svga_block_map *map,
                                        svga_stream_t stream);

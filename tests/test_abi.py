@@ -187,3 +187,48 @@ def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert int(ver) == lib.svga_version() and int(rc) == 0
     assert (int(cls), int(ptr), int(fcap)) == (2 * 3 * 3, 4 * (2 * 3 + 1), 2 * 3 * 3)
     assert bad == "SVGA_ERR_UNSUPPORTED" and "head_dim 96" in r.stdout
+
+
+def test_undersized_plan_is_rejected_on_the_host(lib):
+    """A plan smaller than svga_block_map_size's plan_bytes (the worst case) is refused
+    before any launch by every call that builds or reads a map: a build into it would
+    have to drop entries its items still count, and a kernel reading it would run past
+    its end.  With the full size the same calls get past the map checks."""
+    P = ctypes.c_void_p
+    prob = svga.ProblemSpec.from_workload(C.mid())
+    s = svga.svga_block_map_size(prob)
+    fake = 1 << 20   # aligned, never dereferenced: every call below stops on the host
+
+    def bmap(plan_bytes):
+        return svga.BlockMapC(fake, fake, fake, fake, fake, s["full_cap"], s["bnd_cap"], fake,
+                              plan_bytes, None)
+
+    small = bmap(s["plan_bytes"] - 4)
+    st = P(0)
+    assert lib.svga_build_block_map(ctypes.byref(prob.c), ctypes.byref(small), P(fake),
+                                    s["workspace_bytes"], st) == 5
+    assert b"plan" in lib.svga_last_error()
+    assert lib.svga_build_block_map_static(ctypes.byref(prob.c), ctypes.byref(small), st) == 5
+    wsp = (ctypes.c_int32 * prob.heads)(*([2] * prob.heads))
+    assert lib.svga_build_block_map_routed(ctypes.byref(prob.c), P(fake), wsp, wsp,
+                                           ctypes.byref(small), P(fake), s["workspace_bytes"],
+                                           st) == 5
+    assert lib.svga_sparse_attention_fwd(P(fake), P(fake), P(fake), P(fake), None,
+                                         ctypes.byref(prob.c), ctypes.byref(small),
+                                         ctypes.c_float(0.1), 0, st) == 1
+    assert b"smaller than svga_block_map_size" in lib.svga_last_error()
+    assert lib.svga_permute_tokens_mapped(P(fake), P(1 << 32), ctypes.byref(prob.c),
+                                          ctypes.byref(small), st) == 1
+    assert lib.svga_unpermute_tokens_mapped(P(fake), P(1 << 32), ctypes.byref(prob.c),
+                                            ctypes.byref(small), st) == 1
+    # a misaligned plan is refused too
+    mis = svga.BlockMapC(fake, fake, fake, fake, fake, 0, 0, fake + 16, s["plan_bytes"], None)
+    assert lib.svga_sparse_attention_fwd(P(fake), P(fake), P(fake), P(fake), None,
+                                         ctypes.byref(prob.c), ctypes.byref(mis),
+                                         ctypes.c_float(0.1), 0, st) == 3
+    # the full size passes the map checks and stops at the next host check (the scale)
+    full = bmap(s["plan_bytes"])
+    assert lib.svga_sparse_attention_fwd(P(fake), P(fake), P(fake), P(fake), None,
+                                         ctypes.byref(prob.c), ctypes.byref(full),
+                                         ctypes.c_float(-1.0), 0, st) == 1
+    assert b"scale" in lib.svga_last_error()
