@@ -9,31 +9,39 @@
 // ainews.tenesys.com, "Co sie zmienilo?" items 1-2), written for Blackwell:
 //
 //   * one CTA per work item = two consecutive 128-row query blocks (Q0, Q1) that share
-//     one stream of key chunks (the merged lists of the two blocks);
+//     one stream of key chunks (the merged lists of the two blocks); a visit is one
+//     (chunk, block) pair the block's list holds, taken chunk by chunk, Q0 before Q1;
 //   * warp 0 streams K and V chunks with TMA (128-byte swizzle) through a ring of
-//     shared-memory stages; warp 1 issues tcgen05.mma from one thread:
-//       S_i = Q_i K^T  (A, B from shared memory, D in TMEM, fp32)
-//       O_i += P_i V   (A = P from TMEM as bf16, B = V from shared memory)
-//     in the order S0(n+1) after PV0(n) and S1(n+1) after PV1(n), so the two softmax
-//     warpgroups work on different tiles while the tensor core runs the other's MMAs;
-//     operand descriptors are built once and advanced by constant offsets;
+//     shared-memory stages;
+//   * TMEM: S | P0 | P1 | O0 | O1 (128, 64, 64, 128, 128 columns).  The S tile is shared
+//     by the two groups and P has columns of its own, so the S of the next visit can be
+//     computed as soon as the previous S has been read into registers; a group's next S
+//     does not wait for its P V product (with P written over S it would);
+//   * two threads issue tcgen05.mma: warp 1 the products S = Q_i K^T (A, B from shared
+//     memory, D in TMEM, fp32) visit after visit, warp 3 the products O_i += P_i V
+//     (A = P from TMEM as bf16, B = V from shared memory), each P V right behind the S
+//     two visits ahead of it, where it runs while that S is being read.  Neither waits
+//     for the other; the hazards between the streams go through the softmax barriers;
 //   * warps 4-7 and 8-11 hold one query row per thread (TMEM lane = row): they read S,
 //     run the online softmax in the exp2 domain with packed fp32x2 arithmetic and the
-//     MUFU exponential, write P back into TMEM over S as bf16, and rescale O in TMEM
-//     only when the running maximum grows by more than 2^8 (P stays <= 256 otherwise);
+//     MUFU exponential, and write P as bf16 into their P columns.  The reference maximum
+//     is the exact maximum of the row's first visited tile and is kept: later tiles
+//     need no maximum pass; a tile whose P sum would exceed 2^16 is redone with its own
+//     maximum after O is rescaled in TMEM;
 //   * boundary tiles build a 128-bit keep mask per row from the runs of the key chunk
 //     (at most a few intervals per run), then mask with one select per element;
 //   * the producer/MMA warpgroup gives registers to the softmax warpgroups (setmaxnreg);
-//   * TMEM: S0 | S1 | O0 | O1, 128 columns each (512 allocated);
 //   * a launch may run one part of the plan's items (snake order), so one problem can
 //     be split over several GPUs; the tile-aligned traversal (B3) treats every visited
 //     chunk as full;
 //   * with Q and O frame-major, the softmax threads of a temporal-major head copy their
 //     own Q rows into the swizzled Q tile (frame-major heads keep the TMA load) and
 //     every head writes O and LSE rows back to their frame-major tokens;
-//   * with K and V frame-major, warps 2 and 3 gather the key chunks of a temporal-major
-//     head row by row (16-byte cp.async into the same swizzled stage layout) in place of
-//     warp 0's tile loads.
+//   * with K and V frame-major, warp 2 gathers the key chunks of a temporal-major head
+//     row by row (16-byte cp.async into the same swizzled stage layout) in place of
+//     warp 0's tile loads;
+//   * plan entries are read one step ahead and used only at the next step, so that no
+//     warp waits for a global load in its loop.
 //
 // Every mbarrier wait gives up after about a second: the CTA raises a shared abort
 // flag, drains its MMAs and copies, frees TMEM, writes SVGA_ERR_TIMEOUT to the
@@ -54,13 +62,19 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// a tile's P sum above this (2^16) triggers a new reference maximum; every P then stays
+// below it, far inside the range of bf16 P and of the fp32 sums
+constexpr float kTileSumLimit = 65536.0f;
+
 constexpr uint32_t kNegInfBits = 0xff800000u;
 // Register split: the producer / MMA warpgroup drops to kRegsLow, the two softmax
 // warpgroups rise to kRegsHigh.  128 * kRegsLow + 256 * kRegsHigh must not exceed the
 // 384 * kRegsLaunch registers the CTA is launched with (checked on the host).
 constexpr int kRegsLaunch = 168, kRegsLow = 120, kRegsHigh = 192;
-constexpr int kGatherThreads = 64;  // warps 2 and 3, when K / V rows are gathered
+// TMEM columns: the S tile shared by the two groups, a P tile per group, an O per group
+constexpr uint32_t kTmS = 0, kTmP = 128, kTmO = 256;
+constexpr int kGatherThreads = 32;  // warp 2, when K / V rows are gathered
+constexpr int kGatherRows = kGatherThreads / 8;  // chunk rows one gather step covers
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 struct KParams {
@@ -102,10 +116,12 @@ struct Barriers {
     uint64_t q_full;
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_done[2];
-    uint64_t drain;
+    uint64_t s_full[2];  // [group]: that group's S is in the shared S columns
+    uint64_t s_free;     // the S columns were read into registers by their owner (4 warps)
+    uint64_t s_issued[4];  // [visit % 4]: the S issuer has issued the S of that visit
+    uint64_t p_full[2];  // [group]: P of the group's tile is in its P columns (4 warps)
+    uint64_t o_done[2];  // [group]: the group's last P V product is done
+    uint64_t drain[2];   // abort: [issuer]: the MMAs that issuer started are done
     uint32_t tmem_base;
     int abort;
 };
@@ -116,19 +132,29 @@ struct Item {
     bool valid1, ragged;
     int mode, naive, n_kc;
 
-    __device__ __forceinline__ uint32_t entry(int n) const
+    // Entry n as stored (plan mode: a global load).  A prefetched entry is read with
+    // raw() and passed through fix() only where it is used: an instruction that depends on
+    // the load right after it would hold the warp for the whole load latency.
+    __device__ __forceinline__ uint32_t raw(int n) const
     {
-        if (mode == 0) {
-            uint32_t e = __ldg(ent + n);
-            if (naive) e &= ~(kEntF0 | kEntF1);
-            return e;
-        }
         // dense: every chunk, full except a last one that runs past the final token
         const bool full = !(ragged && n == n_kc - 1);
         uint32_t e = (uint32_t)n | kEntV0 | (full ? kEntF0 : 0u);
         if (valid1) e |= kEntV1 | (full ? kEntF1 : 0u);
+        // plan mode: a predicated load over that value (a select between the two would
+        // wait for the load at once)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.eq.s32 p, %2, 0;\n\t@p ld.global.nc.u32 %0, [%1];\n\t}"
+            : "+r"(e)
+            : "l"(ent + n), "r"(mode));
         return e;
     }
+    // The naive traversal clears the full flags (visit flags and chunk are unchanged).
+    __device__ __forceinline__ uint32_t fix(uint32_t e) const
+    {
+        return (mode == 0 && naive) ? (e & ~(kEntF0 | kEntF1)) : e;
+    }
+    __device__ __forceinline__ uint32_t entry(int n) const { return fix(raw(n)); }
 };
 
 // Plan items (sorted longest first) are dealt to the parts in snake order: in group g of
@@ -319,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     const Item it = make_item(p, KN);
-    // keys of a head in a temporal-major order, read from frame-major K and V: warps 2
-    // and 3 gather the chunk rows instead of the TMA producer
+    // keys of a head in a temporal-major order, read from frame-major K and V: warp 2
+    // gathers the chunk rows instead of the TMA producer
     const bool kv_gather = p.kv_fm && p.mode == 0 && __ldg(p.head_info + it.h).z != ORDER_FM;
 
     if (threadIdx.x == 0) {
@@ -335,7 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bar->p_full[i]), 4);  // one arrival per softmax warp
             mbar_init(smem_u32(&bar->o_done[i]), 1);
         }
-        mbar_init(smem_u32(&bar->drain), 1);
+        mbar_init(smem_u32(&bar->s_free), 4);  // one arrival per softmax warp of the owner
+        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bar->s_issued[i]), 1);
+        mbar_init(smem_u32(&bar->drain[0]), 1);
+        mbar_init(smem_u32(&bar->drain[1]), 1);
         bar->abort = 0;
         fence_barrier_init();
     }
@@ -367,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int issued = 0;
             bool ok = true;
+            uint32_t e_nxt = (!kv_gather && it.E > 0) ? it.raw(0) : 0u;  // one entry ahead
             for (int n = 0; n < (kv_gather ? 0 : it.E) && ok; ++n) {
-                const int kc = (int)(it.entry(n) & kEntChunkMask);
+                const int kc = (int)(e_nxt & kEntChunkMask);
+                e_nxt = it.raw(min(n + 1, it.E - 1));
                 for (int t = 0; t < 2; ++t) {
                     const int idx = 2 * n + t, s = idx % C::kStages, round = idx / C::kStages;
                     if (round > 0 &&
@@ -396,23 +427,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
                                           (idx / C::kStages) & 1);
             }
-        } else if (warp >= 2 && kv_gather) {
+        } else if (warp == 2 && kv_gather) {
             // ---------------------------------------------------- K/V row gather
             // Chunk row r holds the key at position kc * KN + r of the head's order; its
-            // frame-major token is found by walking the order's grid.  Eight threads copy
-            // one 128-byte half row, 16 bytes each, into the 128-byte-swizzled stage (the
+            // frame-major token is found by walking the order's grid.  Eight lanes copy one
+            // 128-byte half row, 16 bytes each, into the 128-byte-swizzled stage (the
             // layout the TMA load gives); rows past the last token are zero-filled.  A
             // stage is handed over once its copies have landed and been made visible to
             // the MMA (async proxy); one stage stays in flight behind the one issued.
-            const int gt = threadIdx.x - 64, u = gt & 7, r0 = gt >> 3;
+            const int u = lane & 7, r0 = lane >> 3;  // rows r0 + kGatherRows * g
             const int korder = __ldg(p.head_info + it.h).z;
             // within a head the row offsets fit 32 bits (at most 2^24 rows of 256 bytes)
             const size_t head_off = (size_t)it.h * p.nk_rows * (D * 2);
             const char *kb = static_cast<const char *>(p.k) + head_off;
             const char *vb = static_cast<const char *>(p.v) + head_off;
-            const uint32_t dst_base = smem_u32(sKV) + r0 * 128 + ((u ^ r0) << 4);
+            const uint32_t dst_base = smem_u32(sKV);
             const int total = 2 * it.E;
-            int tok[KN / 8];
+            int tok[KN / kGatherRows];
             bool ok = true;
             for (int idx = 0; idx < total; ++idx) {
                 const int s = idx % C::kStages, round = idx / C::kStages;
@@ -426,19 +457,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     int f = 0, sx = 0;
                     if (pos0 < p.nk_rows) pos_to_coord(korder, pos0, p.F, p.S, f, sx);
 #pragma unroll
-                    for (int g = 0; g < KN / 8; ++g) {
-                        const int pos = pos0 + 8 * g;
+                    for (int g = 0; g < KN / kGatherRows; ++g) {
+                        const int pos = pos0 + kGatherRows * g;
                         tok[g] = pos < p.nk_rows ? f * p.S + sx : -1;
                         if (korder == ORDER_FM) {
-                            for (sx += 8; sx >= p.S; sx -= p.S) ++f;
+                            for (sx += kGatherRows; sx >= p.S; sx -= p.S) ++f;
                         } else if (korder == ORDER_TM_STRICT) {
-                            for (f += 8; f >= p.F; f -= p.F) ++sx;
+                            for (f += kGatherRows; f >= p.F; f -= p.F) ++sx;
                         } else if (f == 0) {  // the anchor frame leads the order
-                            sx += 8;
-                            if (sx >= p.S && pos + 8 < p.nk_rows)
-                                pos_to_coord(korder, pos + 8, p.F, p.S, f, sx);
+                            sx += kGatherRows;
+                            if (sx >= p.S && pos + kGatherRows < p.nk_rows)
+                                pos_to_coord(korder, pos + kGatherRows, p.F, p.S, f, sx);
                         } else {
-                            for (f += 8; f >= p.F; f -= p.F - 1) ++sx;
+                            for (f += kGatherRows; f >= p.F; f -= p.F - 1) ++sx;
                         }
                     }
                 }
@@ -446,13 +477,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const char *base = (idx & 1) ? vb : kb;
                     const uint32_t dst = dst_base + s * C::kKVBytes;
 #pragma unroll
-                    for (int g = 0; g < KN / 8; ++g) {
+                    for (int g = 0; g < KN / kGatherRows; ++g) {
+                        const int row = r0 + kGatherRows * g;  // swizzle: 16-byte unit ^ row % 8
                         const char *src =
                             base + ((uint32_t)(tok[g] < 0 ? 0 : tok[g]) * (D * 2) + u * 16);
 #pragma unroll
                         for (int c = 0; c < D / 64; ++c)
-                            cp_async_16(dst + c * C::kKVChunk + g * 1024, src + c * 128,
-                                        tok[g] < 0 ? 0u : 16u);
+                            cp_async_16(dst + c * C::kKVChunk + row * 128 + ((u ^ (row & 7)) << 4),
+                                        src + c * 128, tok[g] < 0 ? 0u : 16u);
                     }
                 }
                 cp_async_commit();
@@ -469,8 +501,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 mbar_arrive(smem_u32(&bar->kv_full[(total - 1) % C::kStages]));
             }
-        } else if (warp == 1) {
-            // --------------------------------------------------------- MMA issuer
+        } else if ((warp == 1 || warp == 3) && lane == 0) {
+            // ------------------------------------------------------- MMA issuers
+            // TMEM: S (shared by both groups, kTmS) | P0 | P1 (kTmP + 64 g) | O0 | O1 (kTmO + 128 g)
+            // Two threads issue the tcgen05.mma, each waiting on its own barriers with no
+            // warp-wide votes: warp 1 the S = Q K^T products, warp 3 the O += P V
+            // products.  The two streams touch different TMEM columns, and every hazard
+            // between them goes through a barrier the softmax groups complete (the S
+            // columns are rewritten only after their owner has read them, P only after its
+            // P V product is done), so neither issuer waits for the other: while one waits
+            // or does its bookkeeping the other keeps the tensor pipe fed.
+            const bool s_role = warp == 1;
             constexpr uint32_t idS = idesc_bf16_f32(kBlockM, KN, 0);
             constexpr uint32_t idO = idesc_bf16_f32(kBlockM, D, 1);
             // Descriptors with an empty address field; an operand's start address
@@ -478,89 +519,125 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dK = smem_desc_sw128(0, 16, 1024);
             const uint64_t dV = smem_desc_sw128(0, C::kKVChunk, 1024);
             const uint32_t q_addr = smem_u32(sQ) >> 4, kv_addr = smem_u32(sKV) >> 4;
-            bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->q_full), 0, abort_flag));
+            bool ok = !s_role || mbar_wait(smem_u32(&bar->q_full), 0, abort_flag);
             tc_fence_after();
             const int total = 2 * it.E;
             // TMA completion on the barrier makes the stage visible to the MMA (both async
             // proxy); no tcgen05 fence is needed after these waits.
             auto wait_full = [&](int idx) {
-                return __all_sync(0xffffffffu,
-                                  mbar_wait(smem_u32(&bar->kv_full[idx % C::kStages]),
-                                            (idx / C::kStages) & 1, abort_flag));
-            };
-            auto issue_s = [&](int i, int idx) {
-                const uint64_t a0 = dK + (q_addr + i * (C::kQBytes >> 4));
-                const uint64_t b0 = dK + (kv_addr + (idx % C::kStages) * (C::kKVBytes >> 4));
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + i * 128,
-                           a0 + (uint32_t)(((kk >> 2) * C::kQChunk + (kk & 3) * 32) >> 4),
-                           b0 + (uint32_t)(((kk >> 2) * C::kKVChunk + (kk & 3) * 32) >> 4), idS,
-                           kk > 0 ? 1u : 0u);
-                mma_commit(smem_u32(&bar->s_full[i]));
-            };
-            auto issue_pv = [&](int i, int idx, bool first) {
-                const uint64_t b0 = dV + (kv_addr + (idx % C::kStages) * (C::kKVBytes >> 4));
-#pragma unroll
-                for (int kk = 0; kk < KN / 16; ++kk)
-                    mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
-                           b0 + (uint32_t)(kk * (2048 >> 4)), idO, (!first || kk > 0) ? 1u : 0u);
-                mma_commit(smem_u32(&bar->o_done[i]));
+                return mbar_wait(smem_u32(&bar->kv_full[idx % C::kStages]),
+                                 (idx / C::kStages) & 1, abort_flag);
             };
             auto release = [&](int idx) {
                 if (idx + C::kStages < total)
                     mma_commit(smem_u32(&bar->kv_empty[idx % C::kStages]));
             };
-            int pv0 = 0, pv1 = 0;
-            uint32_t e = it.E > 0 ? it.entry(0) : 0u;
-            if (ok && it.E > 0) {
-                ok = wait_full(0);
-                if (ok && lane == 0) {
-                    if (e & kEntV0) issue_s(0, 0);
-                    if (e & kEntV1) issue_s(1, 0);
-                    release(0);
+            // A cursor over the visits of the item: (entry n, group g) for each group
+            // whose block visits entry n, entries ascending, group 0 before group 1.  It
+            // holds its entry and, already requested, the next one, so that stepping to
+            // the next entry waits for no global load.
+            struct Cursor {
+                int n, g;
+                uint32_t e, e1;
+            };
+            auto last_of_chunk = [](const Cursor &c) { return !(c.g == 0 && (c.e & kEntV1)); };
+            auto advance = [&](Cursor &c) {
+                if (!last_of_chunk(c)) {
+                    c.g = 1;
+                    return;
                 }
-                __syncwarp();
-            }
-            for (int n = 0; ok && n < it.E; ++n) {
-                const bool has_next = n + 1 < it.E;
-                const uint32_t en = has_next ? it.entry(n + 1) : 0u;
-                if (!(ok = wait_full(2 * n + 1))) break;
-                if (e & kEntV0) {
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&bar->p_full[0]), pv0 & 1, abort_flag));
+                ++c.n;
+                c.e = c.e1;
+                // unconditional load from a clamped index: a select on the loaded value
+                // would wait for it here (only visit flags are used from it)
+                c.e1 = it.raw(min(c.n + 1, it.E - 1));
+                c.g = (c.e & kEntV0) ? 0 : 1;  // every entry is visited by some block
+            };
+            Cursor c;
+            c.n = 0;
+            c.e = it.E > 0 ? it.raw(0) : 0u;
+            c.e1 = it.E > 0 ? it.raw(min(1, it.E - 1)) : 0u;
+            c.g = (c.e & kEntV0) ? 0 : 1;
+            int k = 0;              // visits done
+            int need_chunk = -1;    // last entry whose K (or V) stage was waited for
+            int pvn0 = 0, pvn1 = 0;  // P V products issued per group
+            // one loop per role, specialised at compile time (less live state each)
+            auto run = [&](auto role_tag) {
+            constexpr bool kSRole = decltype(role_tag)::value;
+            while (ok && c.n < it.E) {
+                if constexpr (kSRole) {
+                    // S of visit k into the shared S columns, once the owner of visit k-1
+                    // has read its S into registers
+                    if (k > 0 && !(ok = mbar_wait(smem_u32(&bar->s_free), (k - 1) & 1, abort_flag)))
+                        break;
                     tc_fence_after();
-                    if (!ok) break;
-                    if (lane == 0) issue_pv(0, 2 * n + 1, pv0 == 0);
-                    ++pv0;
-                }
-                if (has_next) {
-                    if (!(ok = wait_full(2 * n + 2))) break;
-                    if (lane == 0 && (en & kEntV0)) issue_s(0, 2 * n + 2);
-                }
-                if (e & kEntV1) {
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&bar->p_full[1]), pv1 & 1, abort_flag));
-                    tc_fence_after();
-                    if (!ok) break;
-                    if (lane == 0) issue_pv(1, 2 * n + 1, pv1 == 0);
-                    ++pv1;
-                }
-                if (lane == 0) {
-                    if (has_next) {
-                        if (en & kEntV1) issue_s(1, 2 * n + 2);
-                        release(2 * n + 2);
+                    if (c.n != need_chunk) {
+                        if (!(ok = wait_full(2 * c.n))) break;
+                        need_chunk = c.n;
                     }
-                    release(2 * n + 1);
+                    const uint64_t a0 = dK + (q_addr + c.g * (C::kQBytes >> 4));
+                    const uint64_t b0 =
+                        dK + (kv_addr + ((2 * c.n) % C::kStages) * (C::kKVBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + kTmS,
+                               a0 + (uint32_t)(((kk >> 2) * C::kQChunk + (kk & 3) * 32) >> 4),
+                               b0 + (uint32_t)(((kk >> 2) * C::kKVChunk + (kk & 3) * 32) >> 4),
+                               idS, kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&bar->s_full[c.g]));
+                    if (last_of_chunk(c)) release(2 * c.n);
+                    mbar_arrive(smem_u32(&bar->s_issued[k & 3]));
+                } else {
+                    // O_g += P_g V of visit k, once the group has written P
+                    if (c.n != need_chunk) {
+                        if (!(ok = wait_full(2 * c.n + 1))) break;
+                        need_chunk = c.n;
+                    }
+                    int &pvn = c.g ? pvn1 : pvn0;
+                    ok = mbar_wait(smem_u32(&bar->p_full[c.g]), pvn & 1, abort_flag);
+                    // Behind the S of visit k + 2 in the pipe: the S stream is the chain
+                    // (each S waits until the previous one was read), and a P V product
+                    // issued right after an S runs while that S is being read.
+                    // The S of visit m completes phase m / 4 of s_issued[m % 4].  While
+                    // this P V is not issued, the S of visit k + 5 cannot be: an S waits
+                    // for the previous S to be read, which waits for its group's P
+                    // columns, which wait for that group's previous P V; so at most S of
+                    // visits up to k + 4 are issued, and the barrier of visit k + 2 is at
+                    // most one phase past the one waited for (a parity wait would take a
+                    // barrier two phases ahead for one behind).  (After its last S the S
+                    // issuer arrives for two more visits.)
+                    ok = ok && mbar_wait(smem_u32(&bar->s_issued[(k + 2) & 3]),
+                                         ((k + 2) >> 2) & 1, abort_flag);
+                    tc_fence_after();
+                    if (!ok) break;
+                    const uint64_t b0 =
+                        dV + (kv_addr + ((2 * c.n + 1) % C::kStages) * (C::kKVBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < KN / 16; ++kk)
+                        mma_ts(tmem + kTmO + c.g * 128, tmem + kTmP + c.g * 64 + kk * 8,
+                               b0 + (uint32_t)(kk * (2048 >> 4)), idO,
+                               (pvn != 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(&bar->o_done[c.g]));
+                    if (last_of_chunk(c)) release(2 * c.n + 1);
+                    ++pvn;
                 }
-                __syncwarp();
-                e = en;
+                ++k;
+                advance(c);
+            }
+            };
+            if (s_role)
+                run(std::true_type{});
+            else
+                run(std::false_type{});
+            if (ok && s_role) {  // the last two P V products wait for no later S
+                mbar_arrive(smem_u32(&bar->s_issued[k & 3]));
+                mbar_arrive(smem_u32(&bar->s_issued[(k + 1) & 3]));
             }
             if (!ok) {
-                // Abort: wait for every MMA issued so far before TMEM is freed.
-                if (lane == 0) mma_commit(smem_u32(&bar->drain));
-                __syncwarp();
-                mbar_wait_bounded(smem_u32(&bar->drain), 0);
+                // Abort: wait for every MMA this thread issued before TMEM is freed.
+                const uint32_t drain = smem_u32(s_role ? &bar->drain[0] : &bar->drain[1]);
+                mma_commit(drain);
+                mbar_wait_bounded(drain, 0);
             }
         }
     } else {
@@ -568,8 +645,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         setmaxnreg_inc<kRegsHigh>();
         const int wg = (warp - 4) >> 2, quad = warp & 3, row = quad * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + lane_base + wg * 128;
-        const uint32_t tO = tmem + lane_base + 256 + wg * 128;
+        const uint32_t tS = tmem + lane_base + kTmS;            // shared by both groups
+        const uint32_t tP = tmem + lane_base + kTmP + wg * 64;  // this group's P
+        const uint32_t tO = tmem + lane_base + kTmO + wg * 128;
         const int blk = it.b0 + wg;
         const int qpos = blk * kBlockM + row;
         const bool row_valid = qpos < p.nq_rows;
@@ -616,10 +694,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_used = -INFINITY, l = 0.f;
         int visit = 0;
         bool ok = true;
-        uint32_t e_next = it.E > 0 ? it.entry(0) : 0u;
+        uint32_t e_next = it.E > 0 ? it.raw(0) : 0u;  // prefetched, fixed where used
         for (int n = 0; n < it.E; ++n) {
-            const uint32_t e = e_next;
-            if (n + 1 < it.E) e_next = it.entry(n + 1);
+            const uint32_t e = it.fix(e_next);
+            e_next = it.raw(min(n + 1, it.E - 1));  // unconditional: see the MMA cursors
             if (!(e & vbit)) continue;
             ok = __all_sync(0xffffffffu,
                             mbar_wait(smem_u32(&bar->s_full[wg]), visit & 1, abort_flag));
@@ -638,15 +716,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 keep_mask<KN>(korder, p.aligned ? MASK_DENSE : type, band, p.anchor, p.F, p.S,
                               p.nk_rows, fq, sq, kc * KN, keep);
             tmem_wait_ld();
+            // S is in registers: the shared S columns may take the next visit's S
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar->s_free));
 
-            // The two instantiations: full tiles carry no mask arithmetic.
-            auto body = [&](auto masked_tag) {
-                constexpr bool kMasked = decltype(masked_tag)::value;
-                if (kMasked) {
+            // Boundary tiles drop the keys their rows do not keep; full tiles skip this and
+            // share the rest of the code (one copy of the exponential loop, which keeps
+            // the loop small enough to stay in the instruction cache with the MMA issuer).
+            if (!full) {
 #pragma unroll
-                    for (int c = 0; c < KN; ++c)
-                        if (!((keep[c >> 5] >> (c & 31)) & 1u)) r[c] = kNegInfBits;
-                }
+                for (int c = 0; c < KN; ++c)
+                    if (!((keep[c >> 5] >> (c & 31)) & 1u)) r[c] = kNegInfBits;
+            }
+            // exact row maximum of the tile, in the exp2 domain
+            auto tile_max = [&]() {
                 float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < KN; c += 8) {
@@ -655,38 +739,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a2 = fmax3(a2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
                     a3 = fmax3(a3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
                 }
-                const float mt = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
-                bool need = false;
-                float m_new;
-                if (m_used == -INFINITY) {
-                    m_used = m_new = mt;  // O holds only zero rows so far: nothing to rescale
-                } else if (mt > m_used + kRescaleThreshold) {
-                    need = true;
-                    m_new = mt;
-                } else {
-                    m_new = m_used;
-                }
-                if (__any_sync(0xffffffffu, need)) {
-                    // O += P V of the previous visit must be complete before O is touched.
-                    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->o_done[wg]),
-                                                           (visit - 1) & 1, abort_flag));
-                    tc_fence_after();
-                    if (!ok) return;
-                    const float fac = need ? fast_exp2(m_used - m_new) : 1.f;
-                    l *= fac;
-                    m_used = m_new;
+                return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+            };
+            // The reference maximum m_used is the exact maximum of the row's first visited
+            // tile and is kept afterwards: softmax is the same for any reference, so later
+            // tiles need no maximum pass.  A tile whose P sum exceeds kTileSumLimit (a
+            // value far above the reference, or an overflow) is done a second time with its
+            // exact maximum as the new reference, after O and the running sum are rescaled;
+            // every P then stays below the limit.
+            if (m_used == -INFINITY) m_used = tile_max();
+            // O += P V of the previous visit reads the P columns this tile writes: it must
+            // be complete first (in steady state it finished long ago)
+            if (visit > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->o_done[wg]),
+                                                       (visit - 1) & 1, abort_flag));
+                tc_fence_after();
+                if (!ok) break;
+            }
+            float lt;
 #pragma unroll 1
-                    for (int j = 0; j < D / 32; ++j) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + j * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
-                        tmem_st32(tO + j * 32, o);
-                    }
-                    tmem_wait_st();
-                }
+            for (int attempt = 0;; ++attempt) {
+                // P = 2^(x sl2 - m_used) of every column, packed to bf16 into this group's
+                // P columns; lt = the tile's sum of P
                 const float ms = (m_used == -INFINITY) ? 0.f : m_used;
                 const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ms, -ms);
                 float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
@@ -705,14 +779,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                             s0 = fadd2(s0, ev);
                         pk[c2] = pack_bf16x2_int(ev.x, ev.y);
                     }
-                    tmem_st16(tS + j * 16, pk);
+                    tmem_st16(tP + j * 16, pk);
                 }
-                l += (s0.x + s0.y) + (s1.x + s1.y);
-            };
-            if (full)
-                body(std::false_type{});
-            else
-                body(std::true_type{});
+                lt = (s0.x + s0.y) + (s1.x + s1.y);
+                const bool need = !(lt <= kTileSumLimit);
+                if (attempt > 0 || !__any_sync(0xffffffffu, need)) break;
+                // rare: O (complete up to the previous visit, see above) is rescaled to the
+                // tile's exact maximum and the tile is done again
+                const float m_new = need ? fmaxf(m_used, tile_max()) : m_used;
+                const float fac = need ? fast_exp2(m_used - m_new) : 1.f;
+                l *= fac;
+                m_used = m_new;
+#pragma unroll 1
+                for (int j = 0; j < D / 32; ++j) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + j * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
+                    tmem_st32(tO + j * 32, o);
+                }
+                tmem_wait_st();
+            }
+            l += lt;
             if (!ok) break;
             tmem_wait_st();
             // every lane's P is in TMEM (wait::st + fence); after the warp-level sync one
