@@ -37,8 +37,8 @@
 //   * with Q and O frame-major, the softmax threads of a temporal-major head copy their
 //     own Q rows into the swizzled Q tile (frame-major heads keep the TMA load) and
 //     every head writes O and LSE rows back to their frame-major tokens;
-//   * with K and V frame-major, warp 2 gathers the key chunks of a temporal-major head
-//     row by row (16-byte cp.async into the same swizzled stage layout) in place of
+//   * with K and V frame-major, warps 0 and 2 gather the key chunks of a temporal-major
+//     head row by row (16-byte cp.async into the same swizzled stage layout) in place of
 //     warp 0's tile loads;
 //   * plan entries are read one step ahead and used only at the next step, so that no
 //     warp waits for a global load in its loop.
@@ -73,7 +73,7 @@ constexpr uint32_t kNegInfBits = 0xff800000u;
 constexpr int kRegsLaunch = 168, kRegsLow = 120, kRegsHigh = 192;
 // TMEM columns: the S tile shared by the two groups, a P tile per group, an O per group
 constexpr uint32_t kTmS = 0, kTmP = 128, kTmO = 256;
-constexpr int kGatherThreads = 32;  // warp 2, when K / V rows are gathered
+constexpr int kGatherThreads = 64;  // warps 0 and 2, when K / V rows are gathered
 constexpr int kGatherRows = kGatherThreads / 8;  // chunk rows one gather step covers
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
@@ -96,6 +96,13 @@ struct KParams {
     void *o;
     float *lse;
     int32_t *status;
+    // Key-range split: each work item runs as ksplit CTAs, CTA part r taking the item's
+    // entries [r E / ksplit, (r + 1) E / ksplit).  With ksplit > 1 a CTA writes its rows'
+    // unnormalised O (fp32) to part_o and (reference maximum, sum) to part_ml, both
+    // indexed [(r * heads + head) * nq_rows + row], for a merge kernel to combine.
+    int ksplit;
+    float *part_o;
+    float2 *part_ml;
 };
 
 template <int D, int KN>
@@ -131,6 +138,7 @@ struct Item {
     const uint32_t *ent;
     bool valid1, ragged;
     int mode, naive, n_kc;
+    int n0;  // dense: chunk of this part's first entry (key-range split)
 
     // Entry n as stored (plan mode: a global load).  A prefetched entry is read with
     // raw() and passed through fix() only where it is used: an instruction that depends on
@@ -138,8 +146,9 @@ struct Item {
     __device__ __forceinline__ uint32_t raw(int n) const
     {
         // dense: every chunk, full except a last one that runs past the final token
-        const bool full = !(ragged && n == n_kc - 1);
-        uint32_t e = (uint32_t)n | kEntV0 | (full ? kEntF0 : 0u);
+        const int c = n + n0;
+        const bool full = !(ragged && c == n_kc - 1);
+        uint32_t e = (uint32_t)c | kEntV0 | (full ? kEntF0 : 0u);
         if (valid1) e |= kEntV1 | (full ? kEntF1 : 0u);
         // plan mode: a predicated load over that value (a select between the two would
         // wait for the load at once)
@@ -159,10 +168,11 @@ struct Item {
 
 // Plan items (sorted longest first) are dealt to the parts in snake order: in group g of
 // num_parts consecutive items, part r takes item r when g is even and num_parts-1-r when
-// g is odd, which keeps the parts' total work within one item of each other.
+// g is odd, which keeps the parts' total work within one item of each other.  Under a
+// key-range split the ksplit consecutive CTAs of one item share its g.
 __device__ __forceinline__ int plan_item_of_block(const KParams &p)
 {
-    const int g = blockIdx.x, r = p.part, n = p.num_parts;
+    const int g = blockIdx.x / p.ksplit, r = p.part, n = p.num_parts;
     return g * n + ((g & 1) ? n - 1 - r : r);
 }
 
@@ -197,18 +207,27 @@ __device__ __forceinline__ Item make_item(const KParams &p, int kn)
     it.naive = p.naive;
     it.n_kc = p.n_kc;
     it.ragged = (p.nk_rows % kn) != 0;
+    int e_all;  // entries of the whole item
     if (p.mode == 0) {
         const int4 x = __ldg(p.items + plan_item_of_block(p));
         it.h = x.x;
         it.b0 = x.y;
         it.ent = p.entries + x.z;
-        it.E = x.w;
+        e_all = x.w;
     } else {
-        it.h = blockIdx.x / p.n_pairs;
-        it.b0 = 2 * (blockIdx.x - it.h * p.n_pairs);
+        const int item = blockIdx.x / p.ksplit;
+        it.h = item / p.n_pairs;
+        it.b0 = 2 * (item - it.h * p.n_pairs);
         it.ent = nullptr;
-        it.E = p.n_kc;
+        e_all = p.n_kc;
     }
+    // this CTA's share of the entries (all of them without a key-range split)
+    const int r = blockIdx.x % p.ksplit;
+    const int e0 = (int)((long long)r * e_all / p.ksplit);
+    const int e1 = (int)((long long)(r + 1) * e_all / p.ksplit);
+    if (it.ent) it.ent += e0;
+    it.n0 = e0;
+    it.E = e1 - e0;
     it.valid1 = it.b0 + 1 < p.n_qblk;
     return it;
 }
@@ -345,8 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     const Item it = make_item(p, KN);
-    // keys of a head in a temporal-major order, read from frame-major K and V: warp 2
-    // gathers the chunk rows instead of the TMA producer
+    // keys of a head in a temporal-major order, read from frame-major K and V: warps 0 and
+    // 2 gather the chunk rows instead of the TMA producer's tile loads
     const bool kv_gather = p.kv_fm && p.mode == 0 && __ldg(p.head_info + it.h).z != ORDER_FM;
 
     if (threadIdx.x == 0) {
@@ -427,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
                                           (idx / C::kStages) & 1);
             }
-        } else if (warp == 2 && kv_gather) {
+        }
+        if ((warp == 0 || warp == 2) && kv_gather) {
             // ---------------------------------------------------- K/V row gather
             // Chunk row r holds the key at position kc * KN + r of the head's order; its
             // frame-major token is found by walking the order's grid.  Eight lanes copy one
@@ -435,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // layout the TMA load gives); rows past the last token are zero-filled.  A
             // stage is handed over once its copies have landed and been made visible to
             // the MMA (async proxy); one stage stays in flight behind the one issued.
-            const int u = lane & 7, r0 = lane >> 3;  // rows r0 + kGatherRows * g
+            // warp 0 joins once its lane 0 has issued the Q load (no K / V tile loads then)
+            const int gt = (warp == 0 ? 0 : 32) + lane;
+            const int u = gt & 7, r0 = gt >> 3;  // rows r0 + kGatherRows * g
             const int korder = __ldg(p.head_info + it.h).z;
             // within a head the row offsets fit 32 bits (at most 2^24 rows of 256 bytes)
             const size_t head_off = (size_t)it.h * p.nk_rows * (D * 2);
@@ -817,9 +839,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mbar_wait(smem_u32(&bar->o_done[wg]), (visit - 1) & 1, abort_flag));
             tc_fence_after();
         }
+        // a key-range part (fp32 output only) leaves its rows unnormalised, with their
+        // reference maximum and sum, for the merge
+        const bool split = OUT_F32 && p.part_o != nullptr;
         if (ok && (blk < p.n_qblk)) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t orow = ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * D;
+            const float inv = split ? 1.f : (l > 0.f ? 1.f / l : 0.f);
+            const size_t prow =
+                split ? (size_t)(blockIdx.x % p.ksplit) * p.heads * p.nq_rows : (size_t)0;
+            const size_t orow = (prow + (size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * D;
 #pragma unroll 1
             for (int j = 0; j < D / 32; ++j) {
                 uint32_t o[32];
@@ -832,8 +859,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (row_valid) {
                     if (OUT_F32) {
-                        float4 *dst =
-                            reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + j * 32);
+                        float4 *dst = reinterpret_cast<float4 *>(
+                            (split ? p.part_o : static_cast<float *>(p.o)) + orow + j * 32);
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv,
@@ -856,7 +883,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (row_valid && p.lse)
+            if (row_valid && split)
+                p.part_ml[prow + (size_t)it.h * p.nq_rows + tok] = make_float2(m_used, l);
+            else if (row_valid && p.lse)
                 p.lse[(size_t)it.h * p.nq_rows + tok] =
                     l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
@@ -936,7 +965,8 @@ svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
         set_error("cudaFuncSetAttribute(max dynamic shared memory) failed");
         return SVGA_ERR_CUDA;
     }
-    const int grid = a.mode == 0 ? (a.n_items + kp.num_parts - 1) / kp.num_parts : a.n_items;
+    const int groups = a.mode == 0 ? (a.n_items + kp.num_parts - 1) / kp.num_parts : a.n_items;
+    const int grid = groups * kp.ksplit;
     if (grid > 0) kfn<<<grid, kThreads, C::kSmemLaunch, st>>>(tq, tk, tv, kp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -946,7 +976,64 @@ svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
     return SVGA_OK;
 }
 
+// One thread per 4 output columns of a row: the parts' maxima give the common scale
+// 2^(m_r - m), the weighted sums add in part order (deterministic), and the row is
+// divided by the weighted total.  A part that saw no key of the row has l = 0 and adds
+// nothing.
+__global__ void __launch_bounds__(256) merge_parts_kernel(const float4 *__restrict__ part_o,
+                                                          const float2 *__restrict__ part_ml,
+                                                          int ksplit, size_t rows, int d4,
+                                                          float4 *__restrict__ o)
+{
+    const size_t n = rows * d4;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = i / d4;
+        float m = -INFINITY;
+        for (int r = 0; r < ksplit; ++r) {
+            const float2 ml = __ldg(part_ml + r * rows + row);
+            if (ml.y > 0.f) m = fmaxf(m, ml.x);
+        }
+        float l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < ksplit; ++r) {
+            const float2 ml = __ldg(part_ml + r * rows + row);
+            if (!(ml.y > 0.f)) continue;
+            const float w = exp2f(ml.x - m);
+            const float4 x = __ldg(part_o + r * n + i);
+            l += w * ml.y;
+            acc.x += w * x.x;
+            acc.y += w * x.y;
+            acc.z += w * x.z;
+            acc.w += w * x.w;
+        }
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        o[i] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+}
+
 }  // namespace
+
+svga_status merge_attention_parts(const AttnLaunch &a, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (a.ksplit <= 1) return SVGA_OK;
+    const size_t rows = (size_t)a.heads * a.nq_rows;
+    const int d4 = a.d / 4;
+    const size_t n = rows * d4;
+    const int blocks = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+    if (blocks > 0)
+        merge_parts_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(a.part_o),
+                                                   reinterpret_cast<const float2 *>(a.part_ml),
+                                                   a.ksplit, rows, d4,
+                                                   static_cast<float4 *>(a.o));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error("attention part merge launch failed: %s", cudaGetErrorString(e));
+        return SVGA_ERR_CUDA;
+    }
+    return SVGA_OK;
+}
 
 svga_status launch_attention(const AttnLaunch &a, void *stream)
 {
@@ -996,6 +1083,14 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.o = a.o;
     kp.lse = a.lse;
     kp.status = a.status;
+    const bool split = a.ksplit > 1;
+    if (split && (!a.out_f32 || !a.part_o || !a.part_ml)) {
+        set_error("a key-range split needs fp32 output and part buffers");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    kp.ksplit = split ? a.ksplit : 1;
+    kp.part_o = split ? a.part_o : nullptr;
+    kp.part_ml = split ? reinterpret_cast<float2 *>(a.part_ml) : nullptr;
     const int d = a.d, kn = a.kn;
     if (d == 128 && kn == 128)
         return a.out_f32 ? launch_t<128, 128, true>(a, kp, st) : launch_t<128, 128, false>(a, kp, st);

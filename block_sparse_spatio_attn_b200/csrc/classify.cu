@@ -358,9 +358,36 @@ __global__ void mse_final_kernel(const double *partial, int heads, int n, int32_
     type_out[h] = s <= t ? MASK_SPATIAL : MASK_TEMPORAL;
 }
 
+// Key-range split of the three passes.  With 1% of the rows sampled the passes have few
+// work items (a head and two 128-row blocks each), fewer than the 148 SMs of a B200 at
+// 302,400 tokens and 10 heads (120 items), each with thousands of key chunks.  Splitting
+// every item's chunks over P CTAs (P <= kMaxSplit) that write partial outputs, merged
+// afterwards, fills the GPU: P minimises the waves per unit of work,
+// ceil(items P / 148) / P, the smallest P on a tie.  The choice depends on the item
+// count only, so the workspace size does too; on a part with other SM counts the split
+// is still correct, only less well balanced.
+constexpr int kMaxSplit = 8;
+constexpr int kSplitSms = 148;
+
+int classify_ksplit(int n_items)
+{
+    int best = 1;
+    double best_cost = 1e30;
+    for (int P = 1; P <= kMaxSplit; ++P) {
+        const double waves = (double)(((long long)n_items * P + kSplitSms - 1) / kSplitSms);
+        const double cost = waves / P;
+        if (cost < best_cost - 1e-12) {
+            best_cost = cost;
+            best = P;
+        }
+    }
+    return best;
+}
+
 struct ClassifyLayout {
     size_t plan_s, plan_t, plan_hdr, bounds, bounds_t, cnt, off, rows, rows_t, pos_t, s_hist, qg,
-        qg_t, od, os, ot, partial, types, mse, status, total;
+        qg_t, od, os, ot, part_o, part_ml, partial, types, mse, status, total;
+    int ksplit;
 };
 
 ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
@@ -392,6 +419,10 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
     L.od = take((size_t)heads * n_rows * d * 4);
     L.os = take((size_t)heads * n_rows * d * 4);
     L.ot = take((size_t)heads * n_rows * d * 4);
+    L.ksplit = classify_ksplit(n_items);
+    // shared by the three passes, each merged before the next starts
+    L.part_o = L.ksplit > 1 ? take((size_t)L.ksplit * heads * n_rows * d * 4) : 0;
+    L.part_ml = L.ksplit > 1 ? take((size_t)L.ksplit * heads * n_rows * 8) : 0;
     L.partial = take(sizeof(double) * 2 * kMseParts * heads);
     L.types = take(sizeof(int32_t) * heads);
     L.mse = take(sizeof(float) * 2 * heads);
@@ -514,19 +545,26 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.out_f32 = 1;
     a.n_items = n_items;
     a.status = status;
+    a.ksplit = L.ksplit;
+    a.part_o = L.ksplit > 1 ? reinterpret_cast<float *>(w + L.part_o) : nullptr;
+    a.part_ml = L.ksplit > 1 ? reinterpret_cast<float *>(w + L.part_ml) : nullptr;
     svga_status rc;
+    auto pass = [&]() {
+        svga_status r = launch_attention(a, stream);
+        return r != SVGA_OK ? r : merge_attention_parts(a, stream);
+    };
     a.mode = 1;
     a.o = od;
-    if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
+    if ((rc = pass()) != SVGA_OK) return rc;
     a.mode = 0;  // the masked passes through their plans
     a.plan = plan_s;
     a.o = os;
-    if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
+    if ((rc = pass()) != SVGA_OK) return rc;
     a.plan = plan_t;
     a.q = qg_t;
     a.qrow_tokens = rows_t;
     a.o = ot;
-    if ((rc = launch_attention(a, stream)) != SVGA_OK) return rc;
+    if ((rc = pass()) != SVGA_OK) return rc;
     double *partial = reinterpret_cast<double *>(w + L.partial);
     mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(od, os, ot, pos_t, d, n_rows * d,
                                                            partial);

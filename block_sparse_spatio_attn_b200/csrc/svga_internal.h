@@ -103,8 +103,18 @@ struct AttnLaunch {
     int out_f32;               // o is float32 instead of bf16
     int n_items;
     int32_t *status;
+    // key-range split (out_f32 only): each item runs as ksplit CTAs writing unnormalised
+    // fp32 O to part_o [ksplit][heads][nq_rows][d] and (max, sum) to part_ml
+    // [ksplit][heads][nq_rows]; merge_attention_parts combines them into o.  ksplit <= 1: off.
+    int ksplit;
+    float *part_o;
+    float *part_ml;
 };
 svga_status launch_attention(const AttnLaunch &a, void *stream);
+
+// Combine the ksplit parts of a key-range split launch into normalised fp32 o
+// [heads][nq_rows][d]; a row no part visited reads 0.
+svga_status merge_attention_parts(const AttnLaunch &a, void *stream);
 
 // classify.cu
 size_t classify_workspace_bytes(const svga_problem *p, int n_rows);
