@@ -452,9 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Chunk row r holds the key at position kc * KN + r of the head's order; its
             // frame-major token is found by walking the order's grid.  Eight lanes copy one
             // 128-byte half row, 16 bytes each, into the 128-byte-swizzled stage (the
-            // layout the TMA load gives); rows past the last token are zero-filled.  A
-            // stage is handed over once its copies have landed and been made visible to
-            // the MMA (async proxy); one stage stays in flight behind the one issued.
+            // layout the TMA load gives); rows past the last token are zero-filled.  Each
+            // thread's copies arrive on the stage's barrier when they land, so the gather
+            // never waits for its own copies and keeps every free stage in flight; the MMA
+            // issuers order the landed rows before their reads with a proxy fence.
             // warp 0 joins once its lane 0 has issued the Q load (no K / V tile loads then)
             const int gt = (warp == 0 ? 0 : 32) + lane;
             const int u = gt & 7, r0 = gt >> 3;  // rows r0 + kGatherRows * g
@@ -466,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst_base = smem_u32(sKV);
             const int total = 2 * it.E;
             int tok[KN / kGatherRows];
+            int issued = 0;
             bool ok = true;
             for (int idx = 0; idx < total; ++idx) {
                 const int s = idx % C::kStages, round = idx / C::kStages;
@@ -474,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
+                issued = idx + 1;
                 if (!(idx & 1)) {  // the K stage of a chunk: its rows' tokens
                     const int pos0 = (int)(it.entry(idx >> 1) & kEntChunkMask) * KN + r0;
                     int f = 0, sx = 0;
@@ -509,20 +512,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         src + c * 128, tok[g] < 0 ? 0u : 16u);
                     }
                 }
-                cp_async_commit();
-                if (idx > 0) {
-                    cp_async_wait_group<1>();  // stage idx - 1 has landed
-                    if (!(p.test_stall && idx == 1)) {
-                        fence_proxy_async_smem();
-                        mbar_arrive(smem_u32(&bar->kv_full[(idx - 1) % C::kStages]));
-                    }
-                }
+                // the stage's barrier counts this thread once its copies have landed
+                if (!(p.test_stall && idx == 0))
+                    cp_async_arrive_noinc(smem_u32(&bar->kv_full[s]));
             }
-            cp_async_wait_group<0>();  // nothing in flight when the CTA exits
-            if (ok && total > 0) {
-                fence_proxy_async_smem();
-                mbar_arrive(smem_u32(&bar->kv_full[(total - 1) % C::kStages]));
-            }
+            cp_async_wait_all();  // nothing in flight when the CTA exits
+            if (!ok)  // and no arrival still to come: the stages issued last have completed
+                for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
+                    if (!(p.test_stall && idx == 0))
+                        mbar_wait_bounded(smem_u32(&bar->kv_full[idx % C::kStages]),
+                                          (idx / C::kStages) & 1);
         } else if ((warp == 1 || warp == 3) && lane == 0) {
             // ------------------------------------------------------- MMA issuers
             // TMEM: S (shared by both groups, kTmS) | P0 | P1 (kTmP + 64 g) | O0 | O1 (kTmO + 128 g)
@@ -545,10 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int total = 2 * it.E;
             // TMA completion on the barrier makes the stage visible to the MMA (both async
-            // proxy); no tcgen05 fence is needed after these waits.
+            // proxy); no tcgen05 fence is needed after these waits.  Rows gathered with
+            // cp.async are generic-proxy writes: the proxy fence after the wait orders them
+            // before the MMA's reads.
             auto wait_full = [&](int idx) {
-                return mbar_wait(smem_u32(&bar->kv_full[idx % C::kStages]),
-                                 (idx / C::kStages) & 1, abort_flag);
+                const bool r = mbar_wait(smem_u32(&bar->kv_full[idx % C::kStages]),
+                                         (idx / C::kStages) & 1, abort_flag);
+                if (kv_gather) fence_proxy_async_smem();
+                return r;
             };
             auto release = [&](int idx) {
                 if (idx + C::kStages < total)

@@ -92,16 +92,17 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
                  : "memory");
 }
 
-__device__ __forceinline__ void cp_async_commit()
+// One arrival on the barrier once every cp.async this thread has issued so far has
+// landed; the barrier's expected count includes it (.noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar)
 {
-    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// Wait until at most N of this thread's committed copy groups are still in flight.
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group()
+// Wait until every cp.async this thread has issued has landed.
+__device__ __forceinline__ void cp_async_wait_all()
 {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar)
