@@ -69,6 +69,12 @@ def _load():
             lib.orc_attention_rows_tile_aligned.restype = I
             lib.orc_attention_rows_tile_aligned.argtypes = [P, P, P, I, I, I, ctypes.c_double,
                                                             I, I, I, P, LL, LL, P, I, P, P]
+            lib.orc_position_padded.restype = LL
+            lib.orc_position_padded.argtypes = [I, I, I, I, I, I]
+            lib.orc_order_coords_padded.restype = I
+            lib.orc_order_coords_padded.argtypes = [I, I, I, I, P, P]
+            lib.orc_tile_counts_padded.restype = I
+            lib.orc_tile_counts_padded.argtypes = [I, I, I, I, I, I, I, I, I, P]
             lib.orc_num_threads.restype = I
             lib.orc_num_threads.argtypes = []
             _lib = lib
@@ -104,6 +110,54 @@ def permutation(order: int, F: int, S: int) -> np.ndarray:
     """perm[pos] = frame-major token index held at position `pos` of `order`."""
     fp, sp = order_coords(order, F, S)
     return fp.astype(np.int64) * S + sp
+
+
+def frame_stride(S: int, frame_pad: int) -> int:
+    """Sp: S rounded up to a multiple of frame_pad (S itself when frame_pad is 0)."""
+    return S if frame_pad == 0 else -(-S // frame_pad) * frame_pad
+
+
+def position_padded(order: int, F: int, S: int, Sp: int, f: int, s: int) -> int:
+    """Position of token (f, s) in the padded layout (frame-major frames at stride Sp)."""
+    return _load().orc_position_padded(order, F, S, Sp, f, s)
+
+
+def permutation_padded(order: int, F: int, S: int, Sp: int) -> np.ndarray:
+    """perm[pos] = frame-major token at position `pos` of the padded layout
+    (F * Sp positions), -1 where the position holds no token."""
+    NP = F * Sp
+    fp = np.empty(NP, np.int32)
+    sp = np.empty(NP, np.int32)
+    rc = _load().orc_order_coords_padded(order, F, S, Sp, _ptr(fp), _ptr(sp))
+    if rc != 0:
+        raise ValueError(f"padded layout invalid ({rc})")
+    perm = fp.astype(np.int64) * S + sp
+    perm[fp < 0] = -1
+    return perm
+
+
+def tile_map_padded(type_: int, band: int, anchor: int, order: int, F: int, S: int, Sp: int,
+                    tq: int, tk: int) -> dict:
+    """tile_map of one head in the padded layout: classes and lists over the F * Sp
+    positions, by counting kept elements (positions without a token keep nothing, so a
+    tile holding one is never full)."""
+    NP = F * Sp
+    nq, nk = -(-NP // tq), -(-NP // tk)
+    counts = np.empty(nq * nk, np.int64)
+    rc = _load().orc_tile_counts_padded(type_, band, anchor, order, F, S, Sp, tq, tk,
+                                        _ptr(counts))
+    if rc != 0:
+        raise RuntimeError(f"orc_tile_counts_padded failed ({rc})")
+    cls = np.empty(nq * nk, np.uint8)
+    fptr = np.empty(nq + 1, np.int32)
+    bptr = np.empty(nq + 1, np.int32)
+    fidx = np.empty(nq * nk, np.int32)
+    bidx = np.empty(nq * nk, np.int32)
+    _load().orc_classes_and_lists(_ptr(counts), nq, nk, tq, tk, _ptr(cls), _ptr(fptr),
+                                  _ptr(fidx), _ptr(bptr), _ptr(bidx))
+    return {"counts": counts.reshape(nq, nk), "cls": cls.reshape(nq, nk),
+            "full_ptr": fptr, "full_idx": fidx[: fptr[-1]].copy(),
+            "bnd_ptr": bptr, "bnd_idx": bidx[: bptr[-1]].copy(), "n_q": nq, "n_k": nk}
 
 
 def keep(type_: int, band: int, anchor: int, fq: int, sq: int, fk: int, sk: int) -> bool:

@@ -27,7 +27,16 @@
  *     other frames s-major: position S + s*(F-1) + (f-1).  The literal order s*F + f is
  *     kept as the "strict" variant;
  *   - a tile that holds padding (positions >= N) is never full: padded pairs are not kept;
- *   - an empty row gives O = 0 and LSE = -inf.
+ *   - an empty row gives O = 0 and LSE = -inf;
+ *   - the tile-aligned traversal (B3: ainews.tenesys.com, "Co sie zmienilo?" item 4;
+ *     oossa.com, opening paragraph) has two readings, both here: the mask snapped to
+ *     tiles (orc_attention_rows_tile_aligned), and an exact layout in which each frame
+ *     of a frame-major head starts at a multiple of a frame stride Sp >= S (positions
+ *     f * Sp + s, positions f * Sp + s with s >= S hold no token); temporal-major heads
+ *     keep their order and the positions from N on hold no token
+ *     (orc_order_coords_padded, orc_tile_counts_padded).  The padded layout changes
+ *     which pairs share a tile, not which pairs are kept, so its attention is the
+ *     plain one.
  *
  * The attention is the plain definition: for each query row, the masked softmax of
  * scale * q . k over the kept keys, applied to V, computed in double precision from the
@@ -104,6 +113,60 @@ void orc_mask(int type, int band, int anchor, int F, int S, uint8_t *mask)
 
 int orc_tile_counts_range(int type, int band, int anchor, int order, int F, int S,
                           int tq, int tk, long long i0, long long i1, int64_t *counts);
+
+/* The padded layout: position of token (f, s) when frame-major frames are laid out
+ * with stride Sp (Sp >= S); the temporal-major orders are not padded. */
+long long orc_position_padded(int order, int F, int S, int Sp, int f, int s)
+{
+    if (order == ORC_FRAME_MAJOR) return (long long)f * Sp + s;
+    return orc_position(order, F, S, f, s);
+}
+
+/* Coordinates at every position 0 .. F * Sp - 1 of the padded layout, -1 / -1 where a
+ * position holds no token; found by scattering the forward map over all tokens.
+ * Returns 0 if every token lands on its own position inside the range. */
+int orc_order_coords_padded(int order, int F, int S, int Sp, int32_t *f_of_pos,
+                            int32_t *s_of_pos)
+{
+    long long NP = (long long)F * Sp;
+    if (Sp < S) return -2;
+    for (long long i = 0; i < NP; ++i) { f_of_pos[i] = -1; s_of_pos[i] = -1; }
+    for (int f = 0; f < F; ++f)
+        for (int s = 0; s < S; ++s) {
+            long long p = orc_position_padded(order, F, S, Sp, f, s);
+            if (p < 0 || p >= NP || f_of_pos[p] != -1) return -1;
+            f_of_pos[p] = f;
+            s_of_pos[p] = s;
+        }
+    return 0;
+}
+
+/* Kept-element counts of every (q-tile, k-tile) pair of one head in the padded layout
+ * (F * Sp positions, tiles tq x tk over positions, the grid padded to whole tiles);
+ * a position without a token keeps nothing.  counts has n_q * n_k entries. */
+int orc_tile_counts_padded(int type, int band, int anchor, int order, int F, int S, int Sp,
+                           int tq, int tk, int64_t *counts)
+{
+    long long NP = (long long)F * Sp;
+    long long nq = (NP + tq - 1) / tq, nk = (NP + tk - 1) / tk;
+    int32_t *fp = (int32_t *)malloc(sizeof(int32_t) * NP);
+    int32_t *sp = (int32_t *)malloc(sizeof(int32_t) * NP);
+    if (!fp || !sp) { free(fp); free(sp); return -2; }
+    if (orc_order_coords_padded(order, F, S, Sp, fp, sp) != 0) { free(fp); free(sp); return -1; }
+    memset(counts, 0, sizeof(int64_t) * nq * nk);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long i = 0; i < nq; ++i) {
+        int64_t *row = counts + i * nk;
+        for (long long q = i * tq; q < (i + 1) * tq && q < NP; ++q) {
+            if (fp[q] < 0) continue;
+            for (long long k = 0; k < NP; ++k)
+                if (fp[k] >= 0) row[k / tk] += orc_keep(type, band, anchor, fp[q], sp[q], fp[k], sp[k]);
+        }
+    }
+    free(fp);
+    free(sp);
+    return 0;
+}
 
 /* Kept-element count of every (q-tile, k-tile) pair of one head whose tokens are
  * laid out in `order`, on the grid padded to whole tiles (padded pairs not kept).
