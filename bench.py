@@ -396,6 +396,42 @@ def run_svga(args, rank, world, local_rank):
               "kept_fraction": b3_pairs / (H * N * N),
               "tflops_on_kept": 4.0 * d * b3_pairs / (b3_ms * 1e-3) / 1e12}
 
+    # the other reading of B3, exact: frames laid out at a stride of whole tiles (the
+    # problem's frame_pad), so that no tile holds two frames; timed alternately with the
+    # unpadded exact traversal
+    b3_padded = None
+    if wl.tile_q >= 128 and (wl.tokens_per_frame % max(wl.tile_q, wl.tile_k)) != 0:
+        fpad = max(wl.tile_q, wl.tile_k)
+        prob_p = svga.ProblemSpec.from_workload(wl, frame_pad=fpad)
+        bmap_p = svga.build_block_map(prob_p)
+        NPr = prob_p.rows
+        qpp, kpp, vpp, opp = (torch.empty(H, NPr, d, dtype=torch.bfloat16, device=dev)
+                              for _ in range(4))
+        for src, dst in ((qd, qpp), (kd, kpp), (vd, vpp)):
+            svga.svga_permute_tokens(src, dst, prob_p)
+        b2_t, bp_t = [], []
+        for rnd in range(4):
+            for padded in ((False, True) if rnd % 2 == 0 else (True, False)):
+                if padded:
+                    t = time_it(lambda: svga.svga_sparse_attention_fwd(
+                        qpp, kpp, vpp, opp, None, prob_p, bmap_p, scale), max(3, reps // 2))
+                else:
+                    t = time_it(lambda: svga.svga_sparse_attention_fwd(
+                        qp, kp, vp, op, None, prob, bmap, scale), max(3, reps // 2))
+                (bp_t if padded else b2_t).append(t)
+        if bmap_p.device_status() != 0:
+            raise RuntimeError(f"device status {bmap_p.device_status()} (padded layout)")
+        nqp, nkp = -(-NPr // wl.tile_q), -(-NPr // wl.tile_k)
+        cls_p = bmap_p.cls[: H * nqp * nkp].view(H, nqp, nkp).cpu()
+        b3_padded = {"ms": statistics.median(bp_t),
+                     "exact_b2_ms_alternating": statistics.median(b2_t),
+                     "frame_pad": fpad, "rows_per_head": NPr,
+                     "visited_tiles": int((cls_p != 0).sum()),
+                     "boundary_tiles": int((cls_p == 2).sum()),
+                     "visited_tiles_unpadded": int((cls != 0).sum()),
+                     "boundary_tiles_unpadded": int((cls == 2).sum())}
+        del qpp, kpp, vpp, opp, bmap_p
+
     # -------- end to end through the public API, host buffers ---------------------
     # Pipelined as a serving loop would run it: step i's inputs are copied in on one
     # stream while step i-1 computes on another, and outputs go out on a third; two sets
@@ -483,7 +519,7 @@ def run_svga(args, rank, world, local_rank):
         "boundary_fraction": boundary / (H * nq * nk),
         "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
         "sparse_over_dense": attn_ms / dense_ms, "target_ratio": kept_frac + 0.15,
-        "naive_b1_ms": naive_ms, "tile_aligned_b3": b3,
+        "naive_b1_ms": naive_ms, "tile_aligned_b3": b3, "tile_aligned_b3_padded": b3_padded,
         "step_with_separate_permutes": {"ms": step_sep_ms, "step_ms_same_conditions": step_ref_ms},
         "step_all_frame_major": {"ms": step_fm_ms, "step_ms_same_conditions": step_ref_ms,
                                  "launches": 1,

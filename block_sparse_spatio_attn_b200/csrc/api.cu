@@ -69,14 +69,26 @@ static svga_status validate_shape(const svga_problem *p, Geometry *g, int heads_
         set_error("tile %dx%d unsupported (64, 128 or 256)", p->tile_q, p->tile_k);
         return SVGA_ERR_UNSUPPORTED;
     }
+    const int tmax = p->tile_q > p->tile_k ? p->tile_q : p->tile_k;
+    if (p->frame_pad < 0 || p->frame_pad > 65536 || (p->frame_pad % tmax) != 0) {
+        set_error("frame_pad %d must be 0 or a multiple of max(tile_q, tile_k) = %d up to 65536",
+                  p->frame_pad, tmax);
+        return SVGA_ERR_INVALID_ARG;
+    }
+    const long long Sp = p->frame_pad ? (S + p->frame_pad - 1) / p->frame_pad * p->frame_pad : S;
+    const long long NP = Sp * p->num_frames;  // positions per head
+    if (NP > kMaxTokens) {
+        set_error("padded positions %lld (frames x %lld) above %d", NP, Sp, kMaxTokens);
+        return SVGA_ERR_SHAPE;
+    }
     {
         // the CSR offsets and the plan's entry offsets are int32: the tile count (the
         // lists' capacity) and the plan's entry capacity must fit
-        const long long tiles = (long long)p->heads * ((N + p->tile_q - 1) / p->tile_q) *
-                                ((N + p->tile_k - 1) / p->tile_k);
+        const long long tiles = (long long)p->heads * ((NP + p->tile_q - 1) / p->tile_q) *
+                                ((NP + p->tile_k - 1) / p->tile_k);
         const long long kn = p->tile_k < 128 ? p->tile_k : 128;
         const long long entries =
-            (long long)p->heads * (((N + kBlockM - 1) / kBlockM + 1) / 2) * ((N + kn - 1) / kn);
+            (long long)p->heads * (((NP + kBlockM - 1) / kBlockM + 1) / 2) * ((NP + kn - 1) / kn);
         if (tiles > INT32_MAX || entries > INT32_MAX) {
             set_error("problem too large: %lld tiles and %lld plan entries, int32 offsets "
                       "hold at most %d",
@@ -109,15 +121,17 @@ static svga_status validate_shape(const svga_problem *p, Geometry *g, int heads_
     g->F = p->num_frames;
     g->S = (int)S;
     g->N = (int)N;
+    g->Sp = (int)Sp;
+    g->NP = (int)NP;
     g->d = p->head_dim;
     g->tile_q = p->tile_q;
     g->tile_k = p->tile_k;
-    g->n_q = ceil_div(N, p->tile_q);
-    g->n_k = ceil_div(N, p->tile_k);
+    g->n_q = ceil_div(NP, p->tile_q);
+    g->n_k = ceil_div(NP, p->tile_k);
     g->kn = p->tile_k < 128 ? p->tile_k : 128;
-    g->n_qblk = ceil_div(N, kBlockM);
+    g->n_qblk = ceil_div(NP, kBlockM);
     g->n_pairs = ceil_div(g->n_qblk, 2);
-    g->n_kc = ceil_div(N, g->kn);
+    g->n_kc = ceil_div(NP, g->kn);
     g->n_items = g->heads * g->n_pairs;
     return SVGA_OK;
 }
@@ -236,6 +250,19 @@ using namespace svga;
 
 extern "C" {
 
+svga_status svga_problem_rows(const svga_problem *problem, int64_t *rows)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if (!rows) {
+        set_error("rows is NULL");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    *rows = g.NP;
+    return SVGA_OK;
+}
+
 svga_status svga_block_map_size(const svga_problem *problem, size_t *cls_bytes, size_t *ptr_bytes,
                                 int64_t *full_cap, int64_t *bnd_cap, size_t *plan_bytes,
                                 size_t *workspace_bytes)
@@ -295,6 +322,21 @@ svga_status svga_build_block_map_routed(const svga_problem *problem, const int32
                                   head_type_dev, w_spatial, w_temporal);
 }
 
+// src and dst of a permutation must not overlap: the frame-major side has N rows per
+// head, the token-order side NP.
+static svga_status check_no_overlap(const Geometry &g, const void *src, const void *dst,
+                                   int inverse)
+{
+    const size_t fm = (size_t)g.heads * g.N * g.d * 2, pos = (size_t)g.heads * g.NP * g.d * 2;
+    const size_t sb = inverse ? pos : fm, db = inverse ? fm : pos;
+    const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
+    if (s < d + db && d < s + sb) {
+        set_error("src and dst overlap");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    return SVGA_OK;
+}
+
 static svga_status permute_common(const void *src, void *dst, const svga_problem *problem,
                                   svga_stream_t stream, int inverse)
 {
@@ -303,12 +345,7 @@ static svga_status permute_common(const void *src, void *dst, const svga_problem
     if (rc != SVGA_OK) return rc;
     if ((rc = check_tensor(src, "src")) != SVGA_OK || (rc = check_tensor(dst, "dst")) != SVGA_OK)
         return rc;
-    const size_t bytes = (size_t)g.heads * g.N * g.d * 2;
-    const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
-    if (s < d + bytes && d < s + bytes) {
-        set_error("src and dst overlap");
-        return SVGA_ERR_INVALID_ARG;
-    }
+    if ((rc = check_no_overlap(g, src, dst, inverse)) != SVGA_OK) return rc;
     return launch_permute(src, dst, problem, g, inverse, stream);
 }
 
@@ -322,12 +359,7 @@ static svga_status permute_mapped_common(const void *src, void *dst, const svga_
     if ((rc = check_map_plan(g, map)) != SVGA_OK) return rc;
     if ((rc = check_tensor(src, "src")) != SVGA_OK || (rc = check_tensor(dst, "dst")) != SVGA_OK)
         return rc;
-    const size_t bytes = (size_t)g.heads * g.N * g.d * 2;
-    const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
-    if (s < d + bytes && d < s + bytes) {
-        set_error("src and dst overlap");
-        return SVGA_ERR_INVALID_ARG;
-    }
+    if ((rc = check_no_overlap(g, src, dst, inverse)) != SVGA_OK) return rc;
     return launch_permute(src, dst, problem, g, inverse, stream, map->plan, map->status);
 }
 
@@ -387,6 +419,15 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
         set_error("SVGA_FLAG_NAIVE_B1 and SVGA_FLAG_TILE_ALIGNED exclude each other");
         return SVGA_ERR_INVALID_ARG;
     }
+    if ((flags & (SVGA_FLAG_QO_FRAME_MAJOR | SVGA_FLAG_KV_FRAME_MAJOR |
+                  SVGA_FLAG_TILE_ALIGNED)) &&
+        g.Sp != g.S) {
+        // the padded layout is the other reading of the tile-aligned traversal
+        set_error("frame-major q / o or k / v and the snapped tile-aligned mask need "
+                  "frame_pad = 0 (got %d)",
+                  problem->frame_pad);
+        return SVGA_ERR_UNSUPPORTED;
+    }
     if ((flags & SVGA_FLAG_TILE_ALIGNED) && problem->tile_q < kBlockM) {
         // a 128-row query block would hold two query tiles with different key sets
         set_error("SVGA_FLAG_TILE_ALIGNED needs tile_q >= %d (got %d)", kBlockM, problem->tile_q);
@@ -406,11 +447,13 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     a.o = o;
     a.lse = lse;
     a.heads = g.heads;
-    a.nq_rows = g.N;
-    a.nk_rows = g.N;
+    a.nq_rows = g.NP;
+    a.nk_rows = g.NP;
     a.d = g.d;
     a.F = g.F;
     a.S = g.S;
+    a.N = g.N;
+    a.Sp = g.Sp;
     a.anchor = problem->anchor_frame0;
     a.scale = scale;
     a.mode = 0;

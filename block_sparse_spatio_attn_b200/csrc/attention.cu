@@ -79,6 +79,7 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "regis
 
 struct KParams {
     int heads, nq_rows, nk_rows, F, S, anchor;
+    int N, Sp;  // tokens and frame stride: frame-major frame f starts at position f * Sp
     float scale_log2;
     int mode, naive, aligned, n_pairs, n_qblk, n_kc;
     int n_items, part, num_parts;  // plan mode: this launch runs the items of one part
@@ -184,12 +185,13 @@ __device__ __forceinline__ bool plan_matches(const KParams &p, int kn)
 {
     const int4 *h4 = reinterpret_cast<const int4 *>(p.hdr);
     // {magic, heads, tokens, frames}, {tokens_per_frame, anchor, tile_q, tile_k},
-    // {kn, n_qblk, n_kc, n_items}, {entry_cap (low, high), reserved}
+    // {kn, n_qblk, n_kc, n_items}, {entry_cap (low, high), frame stride, reserved}
     const int4 a = __ldg(h4), b = __ldg(h4 + 1), c = __ldg(h4 + 2), d = __ldg(h4 + 3);
     const long long entry_cap = (long long)(uint32_t)d.x | ((long long)d.y << 32);
-    if (!(a.x == kPlanMagic && a.y == p.heads && a.z == p.nq_rows && a.z == p.nk_rows &&
-          a.w == p.F && b.x == p.S && b.y == p.anchor && b.z == p.tile_q && b.w == p.tile_k &&
-          c.x == kn && c.y == p.n_qblk && c.z == p.n_kc && c.w == p.n_items))
+    if (!(a.x == kPlanMagic && a.y == p.heads && a.z == p.N && a.w == p.F && b.x == p.S &&
+          b.y == p.anchor && b.z == p.tile_q && b.w == p.tile_k && c.x == kn &&
+          c.y == p.n_qblk && c.z == p.n_kc && c.w == p.n_items && d.z == p.Sp &&
+          p.nq_rows == p.F * p.Sp && p.nk_rows == p.nq_rows))
         return false;
     const int4 x = __ldg(p.items + plan_item_of_block(p));
     if (!(x.x >= 0 && x.x < p.heads && x.y >= 0 && !(x.y & 1) && x.y < p.n_qblk && x.z >= 0 &&
@@ -247,41 +249,47 @@ __device__ __forceinline__ void mask_set(uint32_t (&m)[NW], int c0, int c1)
 }
 
 // Keep mask of the key positions [k0, k0 + KN) for one query (fq, sq): bit c is set
-// when key k0 + c exists and the head's mask keeps it.  The positions of a chunk are
-// walked row by row of the order's grid (a frame in frame-major order, an in-frame
-// index in the temporal-major orders); in each row the kept keys form at most two
-// intervals, so the mask costs a handful of integer operations per row.
+// when position k0 + c holds a key and the head's mask keeps it.  The positions of a
+// chunk are walked row by row of the order's grid (a frame in frame-major order, an
+// in-frame index in the temporal-major orders); in each row the kept keys form at most
+// two intervals, so the mask costs a handful of integer operations per row.  Keys end
+// at position N_end (frame-major: F * Sp, temporal-major: the token count); frame f of
+// a frame-major head starts at f * Sp and holds S keys (Sp > S: the padded layout).  A
+// query without a token (q_tok false) keeps nothing.
 template <int KN>
 __device__ __forceinline__ void keep_mask(int order, int type, int band, int anchor, int F, int S,
-                                          int N, int fq, int sq, int k0, uint32_t (&m)[KN / 32])
+                                          int Sp, int N_end, bool q_tok, int fq, int sq, int k0,
+                                          uint32_t (&m)[KN / 32])
 {
 #pragma unroll
     for (int w = 0; w < KN / 32; ++w) m[w] = 0u;
-    const int kend = min(k0 + KN, N);
-    int pos = k0, fixed, row_start, row_len, fbase;
+    if (!q_tok) return;
+    const int kend = min(k0 + KN, N_end);
+    int pos = k0, fixed, row_start, row_len, row_stride, fbase;
     bool f_fixed;
     if (order == ORDER_FM) {
-        fixed = pos / S;
-        row_start = fixed * S;
+        fixed = pos / Sp;
+        row_start = fixed * Sp;
         row_len = S;
+        row_stride = Sp;
         f_fixed = true;
         fbase = 0;
     } else if (order == ORDER_TM_STRICT) {
         fixed = pos / F;
         row_start = fixed * F;
-        row_len = F;
+        row_len = row_stride = F;
         f_fixed = false;
         fbase = 0;
     } else if (pos < S) {
         fixed = 0;
         row_start = 0;
-        row_len = S;
+        row_len = row_stride = S;
         f_fixed = true;
         fbase = 0;
     } else {
         fixed = (pos - S) / (F - 1);
         row_start = S + fixed * (F - 1);
-        row_len = F - 1;
+        row_len = row_stride = F - 1;
         f_fixed = false;
         fbase = 1;
     }
@@ -293,7 +301,9 @@ __device__ __forceinline__ void keep_mask(int order, int type, int band, int anc
         plo = phi = 0;
     };
 #pragma unroll 1
-    while (pos < kend) {
+    while (true) {
+        pos = max(pos, row_start);  // the positions between a padded frame's end and the next
+        if (pos >= kend) break;
         const int b = min(kend, row_start + row_len);
         auto add = [&](int lo, int hi) {
             lo = max(lo, pos);
@@ -327,16 +337,16 @@ __device__ __forceinline__ void keep_mask(int order, int type, int band, int anc
                 if (anchor && fbase == 0) add(row_start, row_start + 1);
             }
         }
-        pos = b;
+        pos = max(pos, b);
         if (order == ORDER_TM && f_fixed) {  // leave the frame-0 block
             f_fixed = false;
             fbase = 1;
             fixed = 0;
             row_start = S;
-            row_len = F - 1;
+            row_len = row_stride = F - 1;
         } else {
             ++fixed;
-            row_start += row_len;
+            row_start += row_stride;
         }
     }
     flush();
@@ -684,13 +694,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             korder = hi.z;
         }
         int fq = 0, sq = 0;
+        bool q_tok = row_valid;  // false: a position of the padded layout without a token
         if (row_valid && type != MASK_DENSE) {
             if (p.qrow_tokens) {
                 const int t = __ldg(p.qrow_tokens + qpos);
                 fq = t / p.S;
                 sq = t - fq * p.S;
+            } else if (korder == ORDER_FM) {
+                fq = qpos / p.Sp;
+                sq = qpos - fq * p.Sp;
+                q_tok = sq < p.S;
             } else {
-                pos_to_coord(korder, qpos, p.F, p.S, fq, sq);
+                q_tok = qpos < p.N;
+                if (q_tok) pos_to_coord(korder, qpos, p.F, p.S, fq, sq);
             }
         }
         // Q and O frame-major: each thread copies its own Q row from the row's frame-major
@@ -739,7 +755,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t keep[KN / 32];
             if (!full)  // mask computed while the TMEM load is in flight
                 keep_mask<KN>(korder, p.aligned ? MASK_DENSE : type, band, p.anchor, p.F, p.S,
-                              p.nk_rows, fq, sq, kc * KN, keep);
+                              p.Sp, korder == ORDER_FM ? p.nk_rows : p.N, q_tok, fq, sq,
+                              kc * KN, keep);
             tmem_wait_ld();
             // S is in registers: the shared S columns may take the next visit's S
             tc_fence_before();
@@ -1047,6 +1064,8 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.nk_rows = a.nk_rows;
     kp.F = a.F;
     kp.S = a.S;
+    kp.N = a.N > 0 ? a.N : a.nk_rows;  // without a padded layout every row is a token
+    kp.Sp = a.Sp > 0 ? a.Sp : a.S;
     kp.anchor = a.anchor;
     kp.scale_log2 = a.scale * kLog2e;
     kp.mode = a.mode;

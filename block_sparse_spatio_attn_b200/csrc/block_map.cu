@@ -52,13 +52,31 @@ __host__ __device__ __forceinline__ uint32_t run_rects(int u0, int u1, int P, bo
     return 5u;
 }
 
-// Tokens at positions [a, b) of `order` (0 <= a < b <= N) as at most 4 rectangles in
-// fixed slots: r[0] the frame-0 part of the anchor-first order, r[1..3] the run's
-// head, middle and tail.  Returns the valid slots as bits.
+// Tokens at positions [a, b) of `order` (0 <= a < b) as at most 4 rectangles in fixed
+// slots: r[0] the frame-0 part of the anchor-first order, r[1..3] the run's head,
+// middle and tail.  Returns the valid slots as bits.  Frame-major frames lie at stride
+// Sp >= S (the padded layout when Sp > S); temporal-major tokens end at N.  *holes is
+// set when a position of [a, b) holds no token.
 __host__ __device__ __forceinline__ uint32_t tile_rects(int order, int a, int b, int F, int S,
-                                                       Rect (&r)[4])
+                                                       int Sp, int N, Rect (&r)[4], bool &holes)
 {
-    if (order == ORDER_FM) return run_rects(a, b, S, true, 0, r[1], r[2], r[3]) << 1;
+    if (order == ORDER_FM) {
+        uint32_t mk = run_rects(a, b, Sp, true, 0, r[1], r[2], r[3]) << 1;
+        if (Sp > S)
+#pragma unroll
+            for (int i = 1; i < 4; ++i)
+                if (((mk >> i) & 1u) && r[i].s1 >= S) {  // the frame's empty tail
+                    holes = true;
+                    r[i].s1 = S - 1;
+                    if (r[i].s0 > r[i].s1) mk &= ~(1u << i);
+                }
+        return mk;
+    }
+    if (b > N) {
+        holes = true;
+        b = N;
+    }
+    if (a >= b) return 0u;
     if (order == ORDER_TM_STRICT) return run_rects(a, b, F, false, 0, r[1], r[2], r[3]) << 1;
     uint32_t mask = 0;  // anchor-first: frame 0 at positions [0, S), then s-major over f >= 1
     if (a < S) {
@@ -150,17 +168,19 @@ __global__ void __launch_bounds__(256) classify_tiles_kernel(Geometry g, int anc
     const int i = blockIdx.x, h = blockIdx.y;
     const int4 hi = head_info[h];
     const int type = hi.x, band = hi.y, order = hi.z;
-    const int qa = i * g.tile_q, qb = min(g.N, qa + g.tile_q);
-    const bool qpad = qa + g.tile_q > g.N;
+    // tiles cover the NP positions; a tile with a position past them or without a token
+    // is never full
+    const int qa = i * g.tile_q, qb = min(g.NP, qa + g.tile_q);
+    bool qpad = qa + g.tile_q > g.NP;
     Rect qr[4];
-    const uint32_t qm = tile_rects(order, qa, qb, g.F, g.S, qr);
+    const uint32_t qm = tile_rects(order, qa, qb, g.F, g.S, g.Sp, g.N, qr, qpad);
     int nf = 0, nb = 0;
     uint8_t *row = cls + ((size_t)h * g.n_q + i) * g.n_k;
     for (int j = threadIdx.x; j < g.n_k; j += blockDim.x) {
-        const int ka = j * g.tile_k, kb = min(g.N, ka + g.tile_k);
-        const bool kpad = ka + g.tile_k > g.N;
+        const int ka = j * g.tile_k, kb = min(g.NP, ka + g.tile_k);
+        bool kpad = ka + g.tile_k > g.NP;
         Rect kr[4];
-        const uint32_t km = tile_rects(order, ka, kb, g.F, g.S, kr);
+        const uint32_t km = tile_rects(order, ka, kb, g.F, g.S, g.Sp, g.N, kr, kpad);
         bool full = !qpad && !kpad, any = false;
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -389,6 +409,7 @@ svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svg
     hdr.n_kc = g.n_kc;
     hdr.n_items = g.n_items;
     hdr.entry_cap = entry_cap;
+    hdr.frame_stride = g.Sp;
     if (types_dev) {
         BandPairs bp;  // 16 KB: travels as kernel parameters
         for (int h = 0; h < g.heads; ++h)

@@ -30,7 +30,8 @@ struct PlanHeader {
     int32_t heads, tokens, frames, tokens_per_frame, anchor;
     int32_t tile_q, tile_k, kn, n_qblk, n_kc, n_items;
     int64_t entry_cap;
-    int32_t reserved[2];
+    int32_t frame_stride;  // Sp: S rounded up to the problem's frame_pad (S without)
+    int32_t reserved;
 };
 static_assert(sizeof(PlanHeader) == 64, "plan header is 64 bytes");
 constexpr int32_t kPlanMagic = 0x53564741;  // "SVGA"
@@ -40,6 +41,7 @@ constexpr uint32_t kEntV0 = 1u << 24, kEntF0 = 1u << 25, kEntV1 = 1u << 26, kEnt
 
 struct Geometry {
     int heads, F, S, N, d;
+    int Sp, NP;  // frame stride and positions per head (S and N without frame_pad)
     int tile_q, tile_k, n_q, n_k;
     int kn, n_qblk, n_pairs, n_kc, n_items;
 };
@@ -87,6 +89,9 @@ struct AttnLaunch {
     float *lse;
     int heads, nq_rows, nk_rows, d;
     int F, S, anchor;
+    // token positions: frame-major heads put frame f at f * Sp (Sp = S unless padded),
+    // temporal-major heads' tokens fill positions 0 .. N-1; other positions hold none
+    int N, Sp;
     float scale;
     int mode;                  // 0 plan, 1 dense (every chunk of every block pair)
     int naive;                 // plan mode: visit full tiles through the masked path

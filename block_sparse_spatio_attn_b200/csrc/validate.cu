@@ -84,6 +84,29 @@ extern "C" svga_status svga_validate_block_map(const svga_problem *problem,
     };
     if (status[0] != 0) return fail("status word set by the build", status[0], 0);
 
+    // head info first: a tile's "holds a position without a token" depends on the order
+    const int4 *hinfo = reinterpret_cast<const int4 *>(head.data() + sizeof(PlanHeader));
+    for (int h = 0; h < g.heads; ++h)
+        if (hinfo[h].x < 0 || hinfo[h].x > 1 || hinfo[h].y < 0 || hinfo[h].z < 0 || hinfo[h].z > 2)
+            return fail("plan head info invalid (head, type)", h, hinfo[h].x);
+    // holes[order][0 / 1][tile]: the q-tile / k-tile holds a position past the NP
+    // positions or one without a token (frame-major: the padding after each frame;
+    // temporal-major: the positions from N on)
+    std::vector<uint8_t> holes[3][2];
+    for (int od = 0; od < 3; ++od)
+        for (int side = 0; side < 2; ++side) {
+            const int t = side ? g.tile_k : g.tile_q, n = side ? g.n_k : g.n_q;
+            holes[od][side].assign(n, 0);
+            for (int i = 0; i < n; ++i)
+                for (long long pos = (long long)i * t; pos < (long long)(i + 1) * t; ++pos) {
+                    const bool tok = pos < g.NP && (od == ORDER_FM ? (pos % g.Sp) < g.S : pos < g.N);
+                    if (!tok) {
+                        holes[od][side][i] = 1;
+                        break;
+                    }
+                }
+        }
+
     // ---- classes and CSR lists
     for (size_t t = 0; t < cls.size(); ++t)
         if (cls[t] > 2) return fail("tile class outside 0..2 at tile", (long long)t, cls[t]);
@@ -101,13 +124,13 @@ extern "C" svga_status svga_validate_block_map(const svga_problem *problem,
     }
     for (size_t r = 0; r < rows; ++r) {
         const uint8_t *row = cls.data() + r * g.n_k;
-        const int i = (int)(r % g.n_q);
-        const bool qpad = (long long)(i + 1) * g.tile_q > g.N;
+        const int i = (int)(r % g.n_q), od = hinfo[r / g.n_q].z;
+        const bool qpad = holes[od][0][i] != 0;
         int nf = 0, nb = 0;
         for (int j = 0; j < g.n_k; ++j) {
             nf += row[j] == 1;
             nb += row[j] == 2;
-            const bool kpad = (long long)(j + 1) * g.tile_k > g.N;
+            const bool kpad = holes[od][1][j] != 0;
             if (row[j] == 1 && (qpad || kpad))
                 return fail("tile holding padding marked full (row, k-tile)", (long long)r, j);
         }
@@ -133,13 +156,9 @@ extern "C" svga_status svga_validate_block_map(const svga_problem *problem,
         hdr.frames != g.F || hdr.tokens_per_frame != g.S ||
         hdr.anchor != problem->anchor_frame0 || hdr.tile_q != g.tile_q ||
         hdr.tile_k != g.tile_k || hdr.kn != g.kn || hdr.n_qblk != g.n_qblk ||
-        hdr.n_kc != g.n_kc || hdr.n_items != g.n_items)
+        hdr.n_kc != g.n_kc || hdr.n_items != g.n_items || hdr.frame_stride != g.Sp)
         return fail("plan header does not match the problem", hdr.magic, hdr.n_items);
-    const int4 *hinfo = reinterpret_cast<const int4 *>(head.data() + sizeof(PlanHeader));
     const int4 *items = hinfo + g.heads;
-    for (int h = 0; h < g.heads; ++h)
-        if (hinfo[h].x < 0 || hinfo[h].x > 1 || hinfo[h].y < 0 || hinfo[h].z < 0 || hinfo[h].z > 2)
-            return fail("plan head info invalid (head, type)", h, hinfo[h].x);
     const long long entry_cap =
         (long long)((map->plan_bytes - plan_header_bytes(g)) / sizeof(uint32_t));
     std::vector<uint8_t> seen(g.n_items, 0);

@@ -28,7 +28,8 @@ FLAG_QO_FRAME_MAJOR = 4
 FLAG_KV_FRAME_MAJOR = 8
 FLAG_TEST_STALL = 1 << 16
 
-EXPORTED = ["svga_block_map_size", "svga_build_block_map", "svga_build_block_map_static",
+EXPORTED = ["svga_problem_rows", "svga_block_map_size", "svga_build_block_map",
+            "svga_build_block_map_static",
             "svga_permute_tokens",
             "svga_unpermute_tokens", "svga_sparse_attention_fwd", "svga_sparse_attention_fwd_part",
             "svga_validate_block_map", "svga_classify_heads_async", "svga_build_block_map_routed",
@@ -52,7 +53,7 @@ class Problem(ctypes.Structure):
                 ("band", ctypes.POINTER(ctypes.c_int32)),
                 ("order", ctypes.POINTER(ctypes.c_int32)),
                 ("anchor_frame0", ctypes.c_int), ("tile_q", ctypes.c_int),
-                ("tile_k", ctypes.c_int)]
+                ("tile_k", ctypes.c_int), ("frame_pad", ctypes.c_int)]
 
 
 class BlockMapC(ctypes.Structure):
@@ -76,6 +77,7 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         PP = ctypes.POINTER(Problem)
+        lib.svga_problem_rows.argtypes = [PP, ctypes.POINTER(ctypes.c_int64)]
         lib.svga_block_map_size.argtypes = [PP, ctypes.POINTER(SZ), ctypes.POINTER(SZ),
                                             ctypes.POINTER(ctypes.c_int64),
                                             ctypes.POINTER(ctypes.c_int64),
@@ -154,9 +156,26 @@ class _Args:
         return _ptr(t)
 
     def tokens(self, problem, **named):
-        """bf16 [heads, tokens, head_dim] tensors of a problem, in argument order."""
+        """bf16 [heads, tokens, head_dim] frame-major tensors, in argument order."""
         shape = (problem.heads, problem.tokens, problem.head_dim)
         return [self.t(t, n, torch.bfloat16, shape) for n, t in named.items()]
+
+    def positions(self, problem, **named):
+        """bf16 [heads, rows, head_dim] tensors in token order (rows = problem.rows:
+        the tokens, or the padded layout's positions), in argument order."""
+        shape = (problem.heads, problem.rows, problem.head_dim)
+        return [self.t(t, n, torch.bfloat16, shape) for n, t in named.items()]
+
+    def attention(self, problem, flags, q, k, v, o, lse):
+        """q, k, v, o and lse of an attention call: in token order, or frame-major
+        where the flags say so."""
+        qo = self.tokens if flags & FLAG_QO_FRAME_MAJOR else self.positions
+        kv = self.tokens if flags & FLAG_KV_FRAME_MAJOR else self.positions
+        pq, po = qo(problem, q=q, o=o)
+        pk, pv = kv(problem, k=k, v=v)
+        n = problem.tokens if flags & FLAG_QO_FRAME_MAJOR else problem.rows
+        pl = self.t(lse, "lse", torch.float32, (problem.heads, n), optional=True)
+        return pq, pk, pv, po, pl
 
     def done(self):
         for name, t in self.seen:
@@ -178,6 +197,7 @@ class ProblemSpec:
     anchor_frame0: int = 1
     tile_q: int = 128
     tile_k: int = 128
+    frame_pad: int = 0
 
     def __post_init__(self):
         H = self.heads
@@ -186,19 +206,27 @@ class ProblemSpec:
         self._od = (ctypes.c_int32 * H)(*self.order)
         self.c = Problem(H, self.num_frames, self.grid_h, self.grid_w, self.head_dim,
                          self._ht, self._bd, self._od, self.anchor_frame0, self.tile_q,
-                         self.tile_k)
+                         self.tile_k, self.frame_pad)
 
     @property
     def tokens(self) -> int:
         return self.num_frames * self.grid_h * self.grid_w
 
+    @property
+    def rows(self) -> int:
+        """Rows per head of a tensor in token order (svga_problem_rows)."""
+        r = ctypes.c_int64()
+        _check(load().svga_problem_rows(ctypes.byref(self.c), ctypes.byref(r)))
+        return r.value
+
     @classmethod
-    def from_workload(cls, wl, head_type=None, order=None, tile_q=None, tile_k=None):
+    def from_workload(cls, wl, head_type=None, order=None, tile_q=None, tile_k=None,
+                      frame_pad=0):
         return cls(wl.heads, wl.frames, wl.grid_h, wl.grid_w, wl.head_dim,
                    list(wl.head_type if head_type is None else head_type), list(wl.band),
                    list(wl.order if order is None else order), wl.anchor_frame0,
                    wl.tile_q if tile_q is None else tile_q,
-                   wl.tile_k if tile_k is None else tile_k)
+                   wl.tile_k if tile_k is None else tile_k, frame_pad)
 
 
 def svga_block_map_size(problem: ProblemSpec) -> dict:
@@ -258,7 +286,8 @@ def svga_validate_block_map(problem: ProblemSpec, bmap: BlockMap, stream=None) -
 def svga_permute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                         stream=None) -> torch.Tensor:
     a = _Args()
-    ps, pd = a.tokens(problem, src=src, dst=dst)
+    ps, = a.tokens(problem, src=src)
+    pd, = a.positions(problem, dst=dst)
     a.done()
     _check(load().svga_permute_tokens(ps, pd, ctypes.byref(problem.c), _stream(stream)))
     return dst
@@ -267,7 +296,8 @@ def svga_permute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSp
 def svga_unpermute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                           stream=None) -> torch.Tensor:
     a = _Args()
-    ps, pd = a.tokens(problem, src=src, dst=dst)
+    ps, = a.positions(problem, src=src)
+    pd, = a.tokens(problem, dst=dst)
     a.done()
     _check(load().svga_unpermute_tokens(ps, pd, ctypes.byref(problem.c), _stream(stream)))
     return dst
@@ -276,8 +306,7 @@ def svga_unpermute_tokens(src: torch.Tensor, dst: torch.Tensor, problem: Problem
 def svga_sparse_attention_fwd(q, k, v, o, lse, problem: ProblemSpec, bmap: BlockMap,
                               scale: float, flags: int = 0, stream=None) -> torch.Tensor:
     a = _Args()
-    pq, pk, pv, po = a.tokens(problem, q=q, k=k, v=v, o=o)
-    pl = a.t(lse, "lse", torch.float32, (problem.heads, problem.tokens), optional=True)
+    pq, pk, pv, po, pl = a.attention(problem, flags, q, k, v, o, lse)
     a.done()
     _check(load().svga_sparse_attention_fwd(pq, pk, pv, po, pl,
                                             ctypes.byref(problem.c), ctypes.byref(bmap.c),
@@ -289,8 +318,7 @@ def svga_sparse_attention_fwd_part(q, k, v, o, lse, problem: ProblemSpec, bmap: 
                                    scale: float, flags: int, part: int, num_parts: int,
                                    stream=None) -> torch.Tensor:
     a = _Args()
-    pq, pk, pv, po = a.tokens(problem, q=q, k=k, v=v, o=o)
-    pl = a.t(lse, "lse", torch.float32, (problem.heads, problem.tokens), optional=True)
+    pq, pk, pv, po, pl = a.attention(problem, flags, q, k, v, o, lse)
     a.done()
     _check(load().svga_sparse_attention_fwd_part(
         pq, pk, pv, po, pl, ctypes.byref(problem.c), ctypes.byref(bmap.c),
@@ -387,7 +415,8 @@ def svga_build_block_map_routed(problem: ProblemSpec, head_type_dev: torch.Tenso
 def svga_permute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                                bmap: BlockMap, stream=None) -> torch.Tensor:
     a = _Args()
-    ps, pd = a.tokens(problem, src=src, dst=dst)
+    ps, = a.tokens(problem, src=src)
+    pd, = a.positions(problem, dst=dst)
     a.done()
     _check(load().svga_permute_tokens_mapped(ps, pd, ctypes.byref(problem.c),
                                              ctypes.byref(bmap.c), _stream(stream)))
@@ -397,7 +426,8 @@ def svga_permute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: Pr
 def svga_unpermute_tokens_mapped(src: torch.Tensor, dst: torch.Tensor, problem: ProblemSpec,
                                  bmap: BlockMap, stream=None) -> torch.Tensor:
     a = _Args()
-    ps, pd = a.tokens(problem, src=src, dst=dst)
+    ps, = a.positions(problem, src=src)
+    pd, = a.tokens(problem, dst=dst)
     a.done()
     _check(load().svga_unpermute_tokens_mapped(ps, pd, ctypes.byref(problem.c),
                                                ctypes.byref(bmap.c), _stream(stream)))

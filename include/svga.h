@@ -120,9 +120,23 @@ enum {
  *   anchor_frame0  1: every query also keeps all keys of frame 0, the anchor
  *                  (aihirek.info, section "A Sparse VideoGen ..."); 0: no anchor
  *   tile_q, tile_k tile size of the block map: 64, 128 or 256 each
- * Lists and plan are indexed with int32: heads * ceil(N/tile_q) * ceil(N/tile_k) and
- * heads * ceil(N/256) * ceil(N/min(tile_k, 128)) must each stay below 2^31
- * (SVGA_ERR_SHAPE otherwise). */
+ *   frame_pad      0, or a multiple of max(tile_q, tile_k) up to 65536: the padded
+ *                  layout, the exact reading of the pages' tile-aligned traversal (B3:
+ *                  ainews.tenesys.com, "Co sie zmienilo?" item 4; oossa.com, opening
+ *                  paragraph: the mask aligned with the tiles the kernel computes).
+ *                  Frame-major heads lay frame f out at positions f*Sp + s with the
+ *                  frame stride Sp = S rounded up to a multiple of frame_pad, so no
+ *                  tile holds two frames; positions f*Sp + s with s >= S hold no token.
+ *                  Temporal-major heads keep their order; positions N and up hold no
+ *                  token.  Every tensor in token order then has NP = F * Sp rows per
+ *                  head (svga_problem_rows), frame-major tensors keep N.  The kept
+ *                  pairs do not change: results equal the unpadded layout's up to the
+ *                  order of the fp32 sums.  A row without a token reads O = 0 and
+ *                  lse = -inf.  SVGA_FLAG_QO_FRAME_MAJOR and SVGA_FLAG_KV_FRAME_MAJOR
+ *                  need frame_pad = 0 (SVGA_ERR_UNSUPPORTED otherwise).
+ * Lists and plan are indexed with int32: heads * ceil(NP/tile_q) * ceil(NP/tile_k) and
+ * heads * ceil(NP/256) * ceil(NP/min(tile_k, 128)) must each stay below 2^31, and
+ * NP <= 2^24 (SVGA_ERR_SHAPE otherwise).  NP = N without padding. */
 typedef struct {
     int heads;
     int num_frames;
@@ -135,7 +149,12 @@ typedef struct {
     int anchor_frame0;
     int tile_q;
     int tile_k;
+    int frame_pad;
 } svga_problem;
+
+/* Rows per head of a tensor in token order (the permuted Q, K, V, O and lse): NP =
+ * num_frames * Sp with frame_pad, N without.  Host-only; per-head arrays not read. */
+SVGA_API svga_status svga_problem_rows(const svga_problem *problem, int64_t *rows);
 
 /* The block map.  DEVICE buffers owned by the caller, sized by svga_block_map_size.
  *   cls       uint8 [heads][n_q][n_k]: 0 = no kept pair (skipped), 1 = every pair
@@ -228,11 +247,13 @@ SVGA_API svga_status svga_validate_block_map(const svga_problem *problem,
  * dst[h, pos] = src[h, t] where pos is the position of frame-major token t in
  * order[h] (spatial heads usually stay frame-major: a plain copy).  The pages move
  * temporal heads to temporal-major order (ainews.tenesys.com, "Co sie zmienilo?"
- * item 5).  src and dst must not overlap.  Bit-exact copy. */
+ * item 5).  src and dst must not overlap.  Bit-exact copy.  With frame_pad, dst has
+ * svga_problem_rows rows per head and its positions without a token are set to 0. */
 SVGA_API svga_status svga_permute_tokens(const void *src, void *dst, const svga_problem *problem,
                                 svga_stream_t stream);
 
-/* Inverse of svga_permute_tokens: dst[h, t] = src[h, pos]. */
+/* Inverse of svga_permute_tokens: dst[h, t] = src[h, pos] (src with
+ * svga_problem_rows rows per head). */
 SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svga_problem *problem,
                                   svga_stream_t stream);
 
@@ -245,10 +266,11 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  * full tiles run without mask arithmetic, boundary tiles are masked element by
  * element (aihirek.info, section "A TPU-kernel kialakitasa ...").  An empty row
  * gives O = 0 and lse = -inf.
- *   q, k, v, o : DEVICE bf16 [heads, tokens, head_dim], every head in order[h]
- *                (q and o frame-major instead with SVGA_FLAG_QO_FRAME_MAJOR, k and v
- *                with SVGA_FLAG_KV_FRAME_MAJOR)
- *   lse        : DEVICE float [heads, tokens] or NULL (frame-major with that flag)
+ *   q, k, v, o : DEVICE bf16 [heads, rows, head_dim], every head in order[h], rows
+ *                = svga_problem_rows (q and o frame-major [heads, tokens, head_dim]
+ *                instead with SVGA_FLAG_QO_FRAME_MAJOR, k and v with
+ *                SVGA_FLAG_KV_FRAME_MAJOR)
+ *   lse        : DEVICE float [heads, rows] or NULL (frame-major with that flag)
  *   map        : built by svga_build_block_map (or _routed / _static) for this problem;
  *                the per-head type, band and order are read from the map's plan.  The
  *                kernel first compares the plan's header (magic, heads, tokens, frames,

@@ -84,6 +84,55 @@ def test_problem_validation(lib, kw, status):
     assert e.value.status == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(frame_pad=-64), 1),
+    (dict(frame_pad=32), 1),                              # not a multiple of the tiles
+    (dict(frame_pad=64, tile_q=128), 1),                  # multiple of 64, not of 128
+    (dict(frame_pad=65536 + 64), 1),
+    # 4,096 tokens per frame at stride 65,536: 1,024 frames hold 2^26 positions
+    (dict(frame_pad=65536, num_frames=1024, grid_h=64, grid_w=64), 2),
+])
+def test_frame_pad_validation(lib, kw, status):
+    with pytest.raises(svga.SvgaError) as e:
+        svga.svga_block_map_size(_bad(lib, **kw))
+    assert e.value.status == status
+
+
+def test_padded_rows_and_sizes(lib):
+    """The padded layout's row count (frames x S rounded up to frame_pad) drives every
+    tile count: headline spatial frames of 3,600 tokens at stride 3,712 (29 tiles of
+    128)."""
+    wl = C.headline()
+    prob = svga.ProblemSpec.from_workload(wl, frame_pad=128)
+    assert prob.rows == 21 * 3712 and prob.tokens == 75600
+    assert svga.ProblemSpec.from_workload(wl).rows == 75600
+    assert svga.ProblemSpec.from_workload(wl, frame_pad=256).rows == 21 * 3840
+    s = svga.svga_block_map_size(prob)
+    nq = 21 * 29
+    assert s["cls_bytes"] == 10 * nq * nq
+    n_items = 10 * ((nq + 1) // 2)
+    hdr = (64 + 16 * (10 + n_items) + 255) // 256 * 256
+    assert s["plan_bytes"] == hdr + 4 * n_items * nq
+
+
+def test_padded_layout_flag_checks(lib):
+    """The padded layout excludes the frame-major q / o and k / v forms and the snapped
+    tile-aligned mask (its other reading): refused on the host."""
+    P = ctypes.c_void_p
+    m = svga.BlockMapC()
+    m.plan, m.plan_bytes, m.status = 4096, 1 << 30, None   # never dereferenced here
+    prob = svga.ProblemSpec.from_workload(C.mid(), frame_pad=128)
+    for flags in (svga.FLAG_QO_FRAME_MAJOR, svga.FLAG_KV_FRAME_MAJOR, svga.FLAG_TILE_ALIGNED):
+        rc = lib.svga_sparse_attention_fwd(P(4096), P(4096), P(4096), P(4096), None,
+                                           ctypes.byref(prob.c), ctypes.byref(m),
+                                           ctypes.c_float(0.1), flags, P(0))
+        assert rc == 4 and b"frame_pad" in lib.svga_last_error(), flags
+    rc = lib.svga_sparse_attention_fwd(P(4096), P(4096), P(4096), P(4096), None,
+                                       ctypes.byref(prob.c), ctypes.byref(m),
+                                       ctypes.c_float(-1.0), svga.FLAG_NAIVE_B1, P(0))
+    assert rc == 1 and b"scale" in lib.svga_last_error()   # accepted up to the last check
+
+
 def test_pointer_validation_before_launch(lib):
     prob = _bad(lib)
     P = ctypes.c_void_p
@@ -155,15 +204,20 @@ int main(void)
 {
     int type[2] = {SVGA_HEAD_SPATIAL, SVGA_HEAD_TEMPORAL}, band[2] = {1, 8};
     int order[2] = {SVGA_ORDER_FRAME_MAJOR, SVGA_ORDER_TEMPORAL_MAJOR};
-    svga_problem p = {2, 3, 8, 8, 64, type, band, order, 1, 64, 64};
+    svga_problem p = {2, 3, 8, 8, 64, type, band, order, 1, 64, 64, 0};
     size_t cls = 0, ptr = 0, plan = 0, ws = 0;
-    int64_t fcap = 0, bcap = 0;
+    int64_t fcap = 0, bcap = 0, rows = 0, rows_pad = 0;
     svga_status rc = svga_block_map_size(&p, &cls, &ptr, &fcap, &bcap, &plan, &ws);
+    svga_status rr = svga_problem_rows(&p, &rows);
+    p.frame_pad = 128;
+    rr = rr == SVGA_OK ? svga_problem_rows(&p, &rows_pad) : rr;
+    p.frame_pad = 0;
     p.head_dim = 96;
     svga_status bad = svga_block_map_size(&p, &cls, &ptr, &fcap, &bcap, &plan, &ws);
-    printf("%d %d %zu %zu %lld %s %s\n", svga_version(), (int)rc, cls, ptr, (long long)fcap,
-           svga_status_string(bad), svga_last_error());
-    return rc == SVGA_OK && bad == SVGA_ERR_UNSUPPORTED ? 0 : 1;
+    printf("%d %d %zu %zu %lld %lld %lld %s %s\n", svga_version(), (int)rc, cls, ptr,
+           (long long)fcap, (long long)rows, (long long)rows_pad, svga_status_string(bad),
+           svga_last_error());
+    return rc == SVGA_OK && rr == SVGA_OK && bad == SVGA_ERR_UNSUPPORTED ? 0 : 1;
 }
 """
 
@@ -183,9 +237,10 @@ def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
-    ver, rc, cls, ptr, fcap, bad = r.stdout.split()[:6]
+    ver, rc, cls, ptr, fcap, rows, rows_pad, bad = r.stdout.split()[:8]
     assert int(ver) == lib.svga_version() and int(rc) == 0
     assert (int(cls), int(ptr), int(fcap)) == (2 * 3 * 3, 4 * (2 * 3 + 1), 2 * 3 * 3)
+    assert (int(rows), int(rows_pad)) == (3 * 64, 3 * 128)   # frames of 64 at stride 128
     assert bad == "SVGA_ERR_UNSUPPORTED" and "head_dim 96" in r.stdout
 
 
