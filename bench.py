@@ -224,6 +224,26 @@ def run_svga(args, rank, world, local_rank):
                            "order": order})
         classify = {"ms": classify_ms, "rows_per_head": n_rows, "types": list(types),
                     "mse": [[round(a, 9), round(b, 9)] for a, b in mse]}
+        if args.mode != "classify":
+            # band selection over a ladder around the classifier's candidates, under the
+            # pages' kept budget (38.87 % of the pairs)
+            cands = [(C.SPATIAL, 2), (C.SPATIAL, 3), (C.SPATIAL, 4),
+                     (C.TEMPORAL, 1200), (C.TEMPORAL, 2400), (C.TEMPORAL, 4800)]
+            ws_at = torch.empty(svga.svga_autotune_size(prob0, n_rows, len(cands)),
+                                dtype=torch.uint8, device=dev)
+            at = svga.svga_autotune_heads(qd, kd, vd, prob0, cands, 0.3887, None, n_rows, scale,
+                                          ws_at)
+            t0 = time.perf_counter()
+            for _ in range(3):
+                at = svga.svga_autotune_heads(qd, kd, vd, prob0, cands, 0.3887, None, n_rows,
+                                              scale, ws_at)
+            classify["band_selection"] = {
+                "ms": (time.perf_counter() - t0) / 3 * 1e3, "candidates": cands,
+                "max_kept_fraction": 0.3887,
+                "kept_fractions": [round(svga.svga_kept_fraction(prob0, t, b), 5)
+                                   for t, b in cands],
+                "types": at[0], "bands": at[1]}
+            del ws_at
         if args.mode == "classify":
             # profiling aid: the classifier alone (Q/K/V and its workspace on the device)
             for _ in range(args.steps):

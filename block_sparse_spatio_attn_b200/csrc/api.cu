@@ -551,7 +551,7 @@ svga_status svga_classify_size(const svga_problem *problem, int n_rows, size_t *
         set_error("n_rows %d outside 1..%d", n_rows, g.N);
         return SVGA_ERR_SHAPE;
     }
-    if (workspace_bytes) *workspace_bytes = classify_workspace_bytes(problem, n_rows);
+    if (workspace_bytes) *workspace_bytes = classify_workspace_bytes(problem, n_rows, 2);
     return SVGA_OK;
 }
 
@@ -585,7 +585,7 @@ static svga_status check_classify(const void *q, const void *k, const void *v,
         return SVGA_ERR_INVALID_ARG;
     }
     if (!workspace || !aligned(workspace, 256) ||
-        workspace_bytes < classify_workspace_bytes(problem, n_rows)) {
+        workspace_bytes < classify_workspace_bytes(problem, n_rows, 2)) {
         set_error("workspace missing, not 256-byte aligned or smaller than svga_classify_size");
         return SVGA_ERR_WORKSPACE;
     }
@@ -621,6 +621,123 @@ svga_status svga_classify_heads_async(const void *q, const void *k, const void *
     }
     return run_classify(q, k, v, problem, w_spatial, w_temporal, rows, n_rows, scale,
                         head_type_dev, mse_dev, status_dev, 1, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Kept (query, key) pairs of one head over the whole problem, counted in closed form
+// from the masks' definitions (every query keeps the keys of frames within `band` of its
+// own, or of in-frame indices within `band` of its own, plus frame 0 with the anchor).
+long long kept_pairs(int type, int band, int anchor, long long F, long long S)
+{
+    if (type == SVGA_HEAD_SPATIAL) {
+        long long frames = 0;  // kept key frames, summed over the query frames
+        for (long long fq = 0; fq < F; ++fq) {
+            const long long lo = fq - band > 0 ? fq - band : 0;
+            const long long hi = fq + band < F - 1 ? fq + band : F - 1;
+            frames += hi - lo + 1 + ((anchor && lo > 0) ? 1 : 0);
+        }
+        return frames * S * S;
+    }
+    long long c = 0;  // kept in-frame pairs (|s_q - s_k| <= band), summed over s_q
+    for (long long sq = 0; sq < S; ++sq) {
+        const long long lo = sq - band > 0 ? sq - band : 0;
+        const long long hi = sq + band < S - 1 ? sq + band : S - 1;
+        c += hi - lo + 1;
+    }
+    return F * (F * c + (anchor ? S * S - c : 0));
+}
+
+}  // namespace
+
+extern "C" {
+
+svga_status svga_kept_fraction(const svga_problem *problem, int head_type, int band,
+                               double *fraction)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if ((head_type != SVGA_HEAD_SPATIAL && head_type != SVGA_HEAD_TEMPORAL) || band < 0 ||
+        band > 65535 || !fraction) {
+        set_error("head_type must be 0 / 1, band 0..65535 and fraction non-NULL");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    const double n = (double)g.N;
+    *fraction = (double)kept_pairs(head_type, band, problem->anchor_frame0, g.F, g.S) / (n * n);
+    return SVGA_OK;
+}
+
+svga_status svga_autotune_size(const svga_problem *problem, int n_rows, int n_cand,
+                               size_t *workspace_bytes)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if (n_rows < 1 || n_rows > g.N || n_cand < 1 || n_cand > max_candidates()) {
+        set_error("n_rows %d outside 1..%d or n_cand %d outside 1..%d", n_rows, g.N, n_cand,
+                  max_candidates());
+        return SVGA_ERR_SHAPE;
+    }
+    if (workspace_bytes) *workspace_bytes = classify_workspace_bytes(problem, n_rows, n_cand);
+    return SVGA_OK;
+}
+
+svga_status svga_autotune_heads(const void *q, const void *k, const void *v,
+                                const svga_problem *problem, const int32_t *cand_type,
+                                const int32_t *cand_band, int n_cand, double max_kept_fraction,
+                                const int32_t *rows, int n_rows, float scale,
+                                int32_t *head_type_out, int32_t *band_out, float *mse_out,
+                                void *workspace, size_t workspace_bytes, svga_stream_t stream)
+{
+    Geometry g;
+    svga_status rc = validate_shape(problem, &g, kHeadsSkip);
+    if (rc != SVGA_OK) return rc;
+    if ((rc = check_tensor(q, "q")) != SVGA_OK || (rc = check_tensor(k, "k")) != SVGA_OK ||
+        (rc = check_tensor(v, "v")) != SVGA_OK)
+        return rc;
+    if (n_rows < 1 || n_rows > g.N || n_cand < 1 || n_cand > max_candidates()) {
+        set_error("n_rows %d outside 1..%d or n_cand %d outside 1..%d", n_rows, g.N, n_cand,
+                  max_candidates());
+        return SVGA_ERR_SHAPE;
+    }
+    if (!cand_type || !cand_band || !head_type_out || !band_out) {
+        set_error("cand_type, cand_band, head_type_out and band_out must be host arrays");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!(max_kept_fraction > 0.0) || !(max_kept_fraction <= 1.0)) {
+        set_error("max_kept_fraction must lie in (0, 1]");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    uint32_t eligible = 0;
+    for (int c = 0; c < n_cand; ++c) {
+        double f = 0.0;
+        if ((rc = svga_kept_fraction(problem, cand_type[c], cand_band[c], &f)) != SVGA_OK)
+            return rc;
+        if (f <= max_kept_fraction) eligible |= 1u << c;
+    }
+    if (!eligible) {
+        set_error("no candidate keeps at most %.6f of the pairs", max_kept_fraction);
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (rows && !aligned(rows, 4)) {
+        set_error("rows is not 4-byte aligned");
+        return SVGA_ERR_ALIGNMENT;
+    }
+    if (!(scale > 0.f) || !(scale < 1e30f)) {
+        set_error("scale must be a positive finite number");
+        return SVGA_ERR_INVALID_ARG;
+    }
+    if (!workspace || !aligned(workspace, 256) ||
+        workspace_bytes < classify_workspace_bytes(problem, n_rows, n_cand)) {
+        set_error("workspace missing, not 256-byte aligned or smaller than svga_autotune_size");
+        return SVGA_ERR_WORKSPACE;
+    }
+    return run_select(q, k, v, problem, n_cand, cand_type, cand_band, eligible, nullptr,
+                      nullptr, rows, n_rows, scale, head_type_out, band_out, mse_out, nullptr, 0,
+                      workspace, workspace_bytes, stream);
 }
 
 const char *svga_last_error(void) { return g_last_error; }

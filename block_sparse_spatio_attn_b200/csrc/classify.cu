@@ -1,21 +1,30 @@
-// classify.cu -- online spatial / temporal head classification.
+// classify.cu -- online spatial / temporal head classification and band selection.
 //
 // Sparse VideoGen profiles the heads while it runs: for a few query rows it computes
 // the dense, the spatial and the temporal outputs and keeps the sparse mask whose
 // output deviates least from the dense one ("Accelerating Spatio-Temporal Attention for
 // Video Diffusion on TPUs", aihirek.info, section "A Sparse VideoGen a figyelmi
-// fejeket osztalyozza").  Here:
-//   1. the sampled rows of Q are gathered into a compact [heads, n_rows, d] tensor;
-//   2. the tcgen05 attention kernel runs three times with the gathered rows as queries
-//      (their original coordinates ride along), writing fp32 outputs: dense over all
-//      keys, then spatial-masked and temporal-masked through small plans of their own:
-//      each 128-row block of sampled rows is bounded by the min / max of its rows'
-//      frame and in-frame index, which decides per key chunk whether it can hold a kept
-//      pair (conservative) and whether every pair is kept (exact), so that the masked
-//      passes skip empty chunks and run full ones unmasked;
-//   3. the two squared deviations are reduced in fp64, first over slices of each head's
-//      outputs by many blocks, then per head in a fixed order (deterministic), and the
-//      smaller one picks the mask (a tie goes to spatial).
+// fejeket osztalyozza").  Here, for a list of candidate masks (type, band):
+//   1. the sampled rows of Q are gathered into a compact [heads, n_rows, d] tensor (and
+//      a second time grouped by in-frame index, for the temporal candidates);
+//   2. the tcgen05 attention kernel runs with the gathered rows as queries (their
+//      original coordinates ride along), writing fp32 outputs: once dense over all
+//      keys, then once per candidate through a small plan of its own: each 128-row block
+//      of sampled rows is bounded by the min / max of its rows' frame and in-frame index,
+//      which decides per key chunk whether it can hold a kept pair (conservative) and
+//      whether every pair is kept (exact), so that a masked pass skips empty chunks and
+//      runs full ones unmasked.  Every pass splits each work item's key range over
+//      several CTAs and merges their partial rows exactly;
+//   3. each candidate's squared deviation from dense is reduced in fp64, first over
+//      slices of each head's outputs by many blocks, then per head in a fixed order
+//      (deterministic), and per head the eligible candidate with the smallest one is
+//      chosen, the earlier candidate on a tie.
+// The classifier proper has two candidates, spatial then temporal, with per-head bands
+// (a tie goes to spatial).  The band selection takes a caller's list of (type, band)
+// candidates; the pages give no rule for trading deviation against cost (the least
+// deviation alone always favours the widest band), so a candidate is eligible when the
+// fraction of pairs its mask keeps stays within a caller's budget, the pages reporting
+// about 39 % of pairs kept (aihirek.info, "A TPU-kernel kialakitasa dontonek bizonyult").
 #include <cuda_runtime.h>
 
 #include "svga_device.cuh"
@@ -29,17 +38,22 @@ struct BandParams {
     uint16_t w_temporal[kMaxHeads];
 };
 
-__global__ void classify_setup_kernel(int heads, int N, int n_rows, int make_rows, BandParams bp,
-                                      int4 *info_s, int4 *info_t, int32_t *rows)
+// The default sampled rows r_i = floor((2i + 1) N / (2 n)) (one per row stratum).
+__global__ void default_rows_kernel(int N, int n_rows, int32_t *rows)
 {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    for (int h = t; h < heads; h += gridDim.x * blockDim.x) {
-        info_s[h] = make_int4(MASK_SPATIAL, bp.w_spatial[h], ORDER_FM, 0);
-        info_t[h] = make_int4(MASK_TEMPORAL, bp.w_temporal[h], ORDER_FM, 0);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows; i += gridDim.x * blockDim.x)
+        rows[i] = (int32_t)(((2ll * i + 1) * (long long)N) / (2ll * n_rows));
+}
+
+// Head info of one candidate's pass plan: its mask type for every head, its band either
+// shared (band >= 0) or per head from the classifier's band arrays (band < 0: the
+// spatial or the temporal array by type); keys stay frame-major.
+__global__ void candidate_info_kernel(int heads, int type, int band, BandParams bp, int4 *info)
+{
+    for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < heads; h += gridDim.x * blockDim.x) {
+        const int b = band >= 0 ? band : (type == MASK_SPATIAL ? bp.w_spatial[h] : bp.w_temporal[h]);
+        info[h] = make_int4(type, b, ORDER_FM, 0);
     }
-    if (make_rows)
-        for (int i = t; i < n_rows; i += gridDim.x * blockDim.x)
-            rows[i] = (int32_t)(((2ll * i + 1) * (long long)N) / (2ll * n_rows));
 }
 
 template <int VPR>
@@ -300,66 +314,72 @@ __global__ void s_scatter_kernel(const int32_t *rows, int n_rows, int N, int S, 
     }
 }
 
-// Stage 1: block (part, h) sums the squared deviations of one slice of head h.  ot holds
-// the temporal pass's rows in the grouped order: row r of od and os is row pos_t[r] there.
-__global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const float *os,
-                                                          const float *ot, const int32_t *pos_t,
-                                                          int d, int n, double *partial)
+// Stage 1: block (part, h) sums the squared deviations of one slice of head h between
+// the dense output od and one candidate's output ox.  With pos (a temporal candidate's
+// pass, which took the rows grouped by in-frame index) row r of od is row pos[r] of ox.
+__global__ void __launch_bounds__(256) mse_partial_kernel(const float *od, const float *ox,
+                                                          const int32_t *pos, int d, int n,
+                                                          double *partial)
 {
-    __shared__ double red[2][8];
+    __shared__ double red[8];
     const int part = blockIdx.x, h = blockIdx.y;
     const size_t base = (size_t)h * n;
     const int per = (n + kMseParts - 1) / kMseParts;
     const int i0 = part * per, i1 = min(n, i0 + per);
-    double as = 0.0, at = 0.0;
+    double acc = 0.0;
     for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
         const int r = i / d, c = i - r * d;
+        const size_t j = pos ? (size_t)__ldg(pos + r) * d + c : (size_t)i;
         const double dv = od[base + i];
-        const double a = os[base + i] - dv;
-        const double b = ot[base + (size_t)__ldg(pos_t + r) * d + c] - dv;
-        as += a * a;
-        at += b * b;
+        const double x = ox[base + j] - dv;
+        acc += x * x;
     }
-    for (int o = 16; o > 0; o >>= 1) {
-        as += __shfl_xor_sync(0xffffffffu, as, o);
-        at += __shfl_xor_sync(0xffffffffu, at, o);
-    }
-    if ((threadIdx.x & 31) == 0) {
-        red[0][threadIdx.x >> 5] = as;
-        red[1][threadIdx.x >> 5] = at;
-    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
     __syncthreads();
     if (threadIdx.x == 0) {
-        double s = 0.0, t = 0.0;
-        for (int w = 0; w < 8; ++w) {
-            s += red[0][w];
-            t += red[1][w];
-        }
-        partial[((size_t)h * kMseParts + part) * 2] = s;
-        partial[((size_t)h * kMseParts + part) * 2 + 1] = t;
+        double t = 0.0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        partial[(size_t)h * kMseParts + part] = t;
     }
 }
 
-// Stage 2: per head, the partial sums in part order, the means and the decision.
-__global__ void mse_final_kernel(const double *partial, int heads, int n, int32_t *type_out,
-                                 float *mse_out)
+constexpr int kMaxCand = 16;  // candidates of one selection
+
+struct CandParams {
+    int n;
+    int type[kMaxCand];
+    int band[kMaxCand];  // shared band, or -1 (per-head bands: no band output)
+    uint32_t eligible;   // bit c: candidate c may be chosen
+};
+
+// Stage 2: per head, each candidate's partial sums in part order (deterministic), its
+// mean, and the choice: the eligible candidate with the least deviation, the earlier
+// one on a tie.
+__global__ void select_kernel(const double *partial, CandParams cp, int heads, int n,
+                              int32_t *type_out, int32_t *band_out, float *mse_out)
 {
     const int h = blockIdx.x * blockDim.x + threadIdx.x;
     if (h >= heads) return;
-    double s = 0.0, t = 0.0;
-    for (int part = 0; part < kMseParts; ++part) {
-        s += partial[((size_t)h * kMseParts + part) * 2];
-        t += partial[((size_t)h * kMseParts + part) * 2 + 1];
+    int best = -1;
+    double best_mse = 0.0;
+    for (int c = 0; c < cp.n; ++c) {
+        const double *pc = partial + ((size_t)c * heads + h) * kMseParts;
+        double t = 0.0;
+        for (int part = 0; part < kMseParts; ++part) t += pc[part];
+        t /= n;
+        mse_out[(size_t)h * cp.n + c] = (float)t;
+        if (((cp.eligible >> c) & 1u) && (best < 0 || t < best_mse)) {
+            best = c;
+            best_mse = t;
+        }
     }
-    s /= n;
-    t /= n;
-    mse_out[2 * h] = (float)s;
-    mse_out[2 * h + 1] = (float)t;
-    type_out[h] = s <= t ? MASK_SPATIAL : MASK_TEMPORAL;
+    type_out[h] = best >= 0 ? cp.type[best] : -1;
+    if (band_out) band_out[h] = best >= 0 ? cp.band[best] : -1;
 }
 
-// Key-range split of the three passes.  With 1% of the rows sampled the passes have few
-// work items (a head and two 128-row blocks each), fewer than the 148 SMs of a B200 at
+// Key-range split of the passes.  With 1% of the rows sampled the passes have few work
+// items (a head and two 128-row blocks each), fewer than the 148 SMs of a B200 at
 // 302,400 tokens and 10 heads (120 items), each with thousands of key chunks.  Splitting
 // every item's chunks over P CTAs (P <= kMaxSplit) that write partial outputs, merged
 // afterwards, fills the GPU: P minimises the waves per unit of work,
@@ -385,12 +405,12 @@ int classify_ksplit(int n_items)
 }
 
 struct ClassifyLayout {
-    size_t plan_s, plan_t, plan_hdr, bounds, bounds_t, cnt, off, rows, rows_t, pos_t, s_hist, qg,
-        qg_t, od, os, ot, part_o, part_ml, partial, types, mse, status, total;
+    size_t plan, plan_hdr, bounds, bounds_t, cnt, off, rows, rows_t, pos_t, s_hist, qg, qg_t, od,
+        ox, part_o, part_ml, partial, types, bands, mse, status, total;
     int ksplit;
 };
 
-ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
+ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S, int n_cand)
 {
     ClassifyLayout L{};
     size_t o = 0;
@@ -399,13 +419,11 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
         o = align_up(o + bytes, 256);
         return at;
     };
-    // the two pass plans, in the attention plan's layout
+    // one pass plan in the attention plan's layout, rebuilt for each candidate
     const int n_qblk = (n_rows + kBlockM - 1) / kBlockM, n_items = heads * ((n_qblk + 1) / 2);
     const int n_kc = (N + 127) / 128;
     L.plan_hdr = align_up(sizeof(PlanHeader) + sizeof(int4) * ((size_t)heads + n_items), 256);
-    const size_t plan_bytes = L.plan_hdr + sizeof(uint32_t) * (size_t)n_items * n_kc;
-    L.plan_s = take(plan_bytes);
-    L.plan_t = take(plan_bytes);
+    L.plan = take(L.plan_hdr + sizeof(uint32_t) * (size_t)n_items * n_kc);
     L.bounds = take(sizeof(int4) * n_qblk);
     L.bounds_t = take(sizeof(int4) * n_qblk);
     L.cnt = take(sizeof(int) * n_items);
@@ -417,15 +435,15 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
     L.qg = take((size_t)heads * n_rows * d * 2);
     L.qg_t = take((size_t)heads * n_rows * d * 2);
     L.od = take((size_t)heads * n_rows * d * 4);
-    L.os = take((size_t)heads * n_rows * d * 4);
-    L.ot = take((size_t)heads * n_rows * d * 4);
+    L.ox = take((size_t)heads * n_rows * d * 4);
     L.ksplit = classify_ksplit(n_items);
-    // shared by the three passes, each merged before the next starts
+    // shared by the passes, each merged before the next starts
     L.part_o = L.ksplit > 1 ? take((size_t)L.ksplit * heads * n_rows * d * 4) : 0;
     L.part_ml = L.ksplit > 1 ? take((size_t)L.ksplit * heads * n_rows * 8) : 0;
-    L.partial = take(sizeof(double) * 2 * kMseParts * heads);
+    L.partial = take(sizeof(double) * (size_t)n_cand * kMseParts * heads);
     L.types = take(sizeof(int32_t) * heads);
-    L.mse = take(sizeof(float) * 2 * heads);
+    L.bands = take(sizeof(int32_t) * heads);
+    L.mse = take(sizeof(float) * (size_t)n_cand * heads);
     L.status = take(sizeof(int32_t));
     L.total = o;
     return L;
@@ -433,27 +451,29 @@ ClassifyLayout classify_layout(int heads, int d, int n_rows, int N, int S)
 
 }  // namespace
 
-size_t classify_workspace_bytes(const svga_problem *p, int n_rows)
+size_t classify_workspace_bytes(const svga_problem *p, int n_rows, int n_cand)
 {
     return classify_layout(p->heads, p->head_dim, n_rows,
-                           p->num_frames * p->grid_h * p->grid_w, p->grid_h * p->grid_w)
+                           p->num_frames * p->grid_h * p->grid_w, p->grid_h * p->grid_w, n_cand)
         .total;
 }
 
-svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
-                         const int32_t *w_spatial, const int32_t *w_temporal, const int32_t *rows,
-                         int n_rows, float scale, int32_t *head_type_out, float *mse_out,
-                         int32_t *status_out, int device_out, void *ws, size_t ws_bytes,
-                         void *stream)
+int max_candidates() { return kMaxCand; }
+
+svga_status run_select(const void *q, const void *k, const void *v, const svga_problem *p,
+                       int n_cand, const int32_t *cand_type, const int32_t *cand_band,
+                       uint32_t eligible, const int32_t *w_spatial, const int32_t *w_temporal,
+                       const int32_t *rows, int n_rows, float scale, int32_t *type_out,
+                       int32_t *band_out, float *mse_out, int32_t *status_out, int device_out,
+                       void *ws, size_t ws_bytes, void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int H = p->heads, d = p->head_dim, S = p->grid_h * p->grid_w, N = p->num_frames * S;
-    const ClassifyLayout L = classify_layout(H, d, n_rows, N, S);
+    const ClassifyLayout L = classify_layout(H, d, n_rows, N, S, n_cand);
     (void)ws_bytes;
     char *w = static_cast<char *>(ws);
-    char *plan_s = w + L.plan_s, *plan_t = w + L.plan_t;
-    int4 *info_s = reinterpret_cast<int4 *>(plan_s + sizeof(PlanHeader));
-    int4 *info_t = reinterpret_cast<int4 *>(plan_t + sizeof(PlanHeader));
+    char *plan = w + L.plan;
+    int4 *info = reinterpret_cast<int4 *>(plan + sizeof(PlanHeader));
     int4 *bounds = reinterpret_cast<int4 *>(w + L.bounds);
     int4 *bounds_t = reinterpret_cast<int4 *>(w + L.bounds_t);
     int32_t *rows_t = reinterpret_cast<int32_t *>(w + L.rows_t);
@@ -465,16 +485,25 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     int32_t *rows_ws = reinterpret_cast<int32_t *>(w + L.rows);
     void *qg = w + L.qg;
     float *od = reinterpret_cast<float *>(w + L.od);
-    float *os = reinterpret_cast<float *>(w + L.os);
-    float *ot = reinterpret_cast<float *>(w + L.ot);
+    float *ox = reinterpret_cast<float *>(w + L.ox);
+    double *partial = reinterpret_cast<double *>(w + L.partial);
     int32_t *types = reinterpret_cast<int32_t *>(w + L.types);
+    int32_t *bands = reinterpret_cast<int32_t *>(w + L.bands);
     float *mse = reinterpret_cast<float *>(w + L.mse);
     int32_t *status = reinterpret_cast<int32_t *>(w + L.status);
 
-    BandParams bp;
-    for (int h = 0; h < H; ++h) {
-        bp.w_spatial[h] = (uint16_t)w_spatial[h];
-        bp.w_temporal[h] = (uint16_t)w_temporal[h];
+    BandParams bp{};
+    if (w_spatial && w_temporal)
+        for (int h = 0; h < H; ++h) {
+            bp.w_spatial[h] = (uint16_t)w_spatial[h];
+            bp.w_temporal[h] = (uint16_t)w_temporal[h];
+        }
+    CandParams cp{};
+    cp.n = n_cand;
+    cp.eligible = eligible;
+    for (int c = 0; c < n_cand; ++c) {
+        cp.type[c] = cand_type[c];
+        cp.band[c] = cand_band ? cand_band[c] : -1;
     }
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess ||
         cudaMemsetAsync(s_hist, 0, sizeof(int) * (size_t)S, st) != cudaSuccess) {
@@ -482,53 +511,36 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         return SVGA_ERR_CUDA;
     }
     const int32_t *rows_use = rows ? rows : rows_ws;
-    classify_setup_kernel<<<(H > n_rows ? H : n_rows) / 256 + 1, 256, 0, st>>>(
-        H, N, n_rows, rows ? 0 : 1, bp, info_s, info_t, rows_ws);
+    if (!rows) default_rows_kernel<<<n_rows / 256 + 1, 256, 0, st>>>(N, n_rows, rows_ws);
     const int vpr = d / 8;
     dim3 grid((n_rows * vpr + 255) / 256 < 1184 ? (n_rows * vpr + 255) / 256 : 1184, H);
-    if (vpr == 16)
-        gather_rows_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
-                                                    static_cast<uint4 *>(qg), rows_use, N, n_rows,
-                                                    status);
-    else
-        gather_rows_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
-                                                   static_cast<uint4 *>(qg), rows_use, N, n_rows,
-                                                   status);
+    auto gather = [&](const int32_t *r, void *dst) {
+        if (vpr == 16)
+            gather_rows_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
+                                                        static_cast<uint4 *>(dst), r, N, n_rows,
+                                                        status);
+        else
+            gather_rows_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
+                                                       static_cast<uint4 *>(dst), r, N, n_rows,
+                                                       status);
+    };
+    gather(rows_use, qg);
     const int n_qblk = (n_rows + kBlockM - 1) / kBlockM, n_pairs = (n_qblk + 1) / 2;
     const int n_items = H * n_pairs, n_kc = (N + 127) / 128;
-    // rows grouped by in-frame index for the temporal pass, its Q rows gathered that way
+    // rows grouped by in-frame index for the temporal passes, their Q rows gathered so
     const int sblocks = (n_rows + 255) / 256 < 1184 ? (n_rows + 255) / 256 : 1184;
     s_hist_kernel<<<sblocks, 256, 0, st>>>(rows_use, n_rows, N, S, s_hist);
     s_scan_kernel<<<1, 1024, 0, st>>>(s_hist, S);
     s_scatter_kernel<<<sblocks, 256, 0, st>>>(rows_use, n_rows, N, S, s_hist, rows_t, pos_t);
-    if (vpr == 16)
-        gather_rows_kernel<16><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
-                                                    static_cast<uint4 *>(qg_t), rows_t, N, n_rows,
-                                                    status);
-    else
-        gather_rows_kernel<8><<<grid, 256, 0, st>>>(static_cast<const uint4 *>(q),
-                                                   static_cast<uint4 *>(qg_t), rows_t, N, n_rows,
-                                                   status);
+    gather(rows_t, qg_t);
     row_bounds_kernel<<<n_qblk, 128, 0, st>>>(rows_use, n_rows, N, S, bounds);
     row_bounds_kernel<<<n_qblk, 128, 0, st>>>(rows_t, n_rows, N, S, bounds_t);
-    for (char *plan : {plan_s, plan_t}) {
-        const int4 *bnd = plan == plan_s ? bounds : bounds_t;
-        int4 *hinfo = reinterpret_cast<int4 *>(plan + sizeof(PlanHeader));
-        int4 *items = hinfo + H;
-        uint32_t *entries = reinterpret_cast<uint32_t *>(plan + L.plan_hdr);
-        pass_count_kernel<<<n_items, 256, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
-                                                   p->anchor_frame0, hinfo, bnd, cnt);
-        pass_items_kernel<<<1, 1024, 0, st>>>(H, n_pairs, n_items, N, n_kc, cnt, off, items, plan);
-        pass_write_kernel<<<n_items, 128, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
-                                                   p->anchor_frame0, hinfo, bnd, off, entries);
-    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("classifier setup launch failed: %s", cudaGetErrorString(e));
         return SVGA_ERR_CUDA;
     }
     AttnLaunch a{};
-    a.q = qg;
     a.k = k;
     a.v = v;
     a.lse = nullptr;
@@ -541,7 +553,6 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
     a.anchor = p->anchor_frame0;
     a.scale = scale;
     a.kn = 128;
-    a.qrow_tokens = rows_use;
     a.out_f32 = 1;
     a.n_items = n_items;
     a.status = status;
@@ -553,33 +564,53 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         svga_status r = launch_attention(a, stream);
         return r != SVGA_OK ? r : merge_attention_parts(a, stream);
     };
+    // the dense pass over every key
     a.mode = 1;
+    a.q = qg;
+    a.qrow_tokens = rows_use;
     a.o = od;
     if ((rc = pass()) != SVGA_OK) return rc;
-    a.mode = 0;  // the masked passes through their plans
-    a.plan = plan_s;
-    a.o = os;
-    if ((rc = pass()) != SVGA_OK) return rc;
-    a.plan = plan_t;
-    a.q = qg_t;
-    a.qrow_tokens = rows_t;
-    a.o = ot;
-    if ((rc = pass()) != SVGA_OK) return rc;
-    double *partial = reinterpret_cast<double *>(w + L.partial);
-    mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(od, os, ot, pos_t, d, n_rows * d,
-                                                           partial);
-    mse_final_kernel<<<(H + 127) / 128, 128, 0, st>>>(partial, H, n_rows * d, types, mse);
+    // one masked pass per candidate through its own plan, and its deviation from dense
+    int4 *items = info + H;
+    uint32_t *entries = reinterpret_cast<uint32_t *>(plan + L.plan_hdr);
+    a.mode = 0;
+    a.plan = plan;
+    a.o = ox;
+    for (int c = 0; c < n_cand; ++c) {
+        const bool temporal = cp.type[c] == MASK_TEMPORAL;
+        const int4 *bnd = temporal ? bounds_t : bounds;
+        candidate_info_kernel<<<H / 256 + 1, 256, 0, st>>>(H, cp.type[c], cp.band[c], bp, info);
+        pass_count_kernel<<<n_items, 256, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
+                                                   p->anchor_frame0, info, bnd, cnt);
+        pass_items_kernel<<<1, 1024, 0, st>>>(H, n_pairs, n_items, N, n_kc, cnt, off, items, plan);
+        pass_write_kernel<<<n_items, 128, 0, st>>>(n_pairs, n_qblk, n_kc, N, S,
+                                                   p->anchor_frame0, info, bnd, off, entries);
+        if ((e = cudaGetLastError()) != cudaSuccess) {
+            set_error("classifier plan launch failed: %s", cudaGetErrorString(e));
+            return SVGA_ERR_CUDA;
+        }
+        a.q = temporal ? qg_t : qg;
+        a.qrow_tokens = temporal ? rows_t : rows_use;
+        if ((rc = pass()) != SVGA_OK) return rc;
+        mse_partial_kernel<<<dim3(kMseParts, H), 256, 0, st>>>(
+            od, ox, temporal ? pos_t : nullptr, d, n_rows * d, partial + (size_t)c * H * kMseParts);
+    }
+    select_kernel<<<(H + 127) / 128, 128, 0, st>>>(partial, cp, H, n_rows * d, types,
+                                                   band_out ? bands : nullptr, mse);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("classifier reduction launch failed: %s", cudaGetErrorString(e));
         return SVGA_ERR_CUDA;
     }
+    const size_t mse_bytes = sizeof(float) * (size_t)n_cand * H;
     if (device_out) {
         // results stay on the device: no host round trip, nothing waits
-        if (cudaMemcpyAsync(head_type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToDevice,
+        if (cudaMemcpyAsync(type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToDevice,
                             st) != cudaSuccess ||
-            (mse_out && cudaMemcpyAsync(mse_out, mse, sizeof(float) * 2 * H,
-                                        cudaMemcpyDeviceToDevice, st) != cudaSuccess) ||
+            (band_out && cudaMemcpyAsync(band_out, bands, sizeof(int32_t) * H,
+                                         cudaMemcpyDeviceToDevice, st) != cudaSuccess) ||
+            (mse_out &&
+             cudaMemcpyAsync(mse_out, mse, mse_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess) ||
             (status_out && cudaMemcpyAsync(status_out, status, sizeof(int32_t),
                                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)) {
             set_error("classifier result copy failed: %s", cudaGetErrorString(cudaGetLastError()));
@@ -588,10 +619,12 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         return SVGA_OK;
     }
     int32_t dev_status = 0;
-    if (cudaMemcpyAsync(head_type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToHost, st) !=
+    if (cudaMemcpyAsync(type_out, types, sizeof(int32_t) * H, cudaMemcpyDeviceToHost, st) !=
             cudaSuccess ||
-        (mse_out && cudaMemcpyAsync(mse_out, mse, sizeof(float) * 2 * H, cudaMemcpyDeviceToHost,
-                                    st) != cudaSuccess) ||
+        (band_out && cudaMemcpyAsync(band_out, bands, sizeof(int32_t) * H, cudaMemcpyDeviceToHost,
+                                     st) != cudaSuccess) ||
+        (mse_out &&
+         cudaMemcpyAsync(mse_out, mse, mse_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
         cudaMemcpyAsync(&dev_status, status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
             cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess) {
@@ -603,6 +636,19 @@ svga_status run_classify(const void *q, const void *k, const void *v, const svga
         return (svga_status)dev_status;
     }
     return SVGA_OK;
+}
+
+svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
+                         const int32_t *w_spatial, const int32_t *w_temporal, const int32_t *rows,
+                         int n_rows, float scale, int32_t *head_type_out, float *mse_out,
+                         int32_t *status_out, int device_out, void *ws, size_t ws_bytes,
+                         void *stream)
+{
+    // two candidates with per-head bands: spatial first, so that a tie goes to spatial
+    const int32_t types[2] = {MASK_SPATIAL, MASK_TEMPORAL};
+    return run_select(q, k, v, p, 2, types, nullptr, 3u, w_spatial, w_temporal, rows, n_rows,
+                      scale, head_type_out, nullptr, mse_out, status_out, device_out, ws, ws_bytes,
+                      stream);
 }
 
 }  // namespace svga

@@ -122,7 +122,17 @@ svga_status launch_attention(const AttnLaunch &a, void *stream);
 svga_status merge_attention_parts(const AttnLaunch &a, void *stream);
 
 // classify.cu
-size_t classify_workspace_bytes(const svga_problem *p, int n_rows);
+size_t classify_workspace_bytes(const svga_problem *p, int n_rows, int n_cand);
+int max_candidates();
+// Dense pass, then one masked pass per candidate (type, band: shared, or per head from
+// w_spatial / w_temporal when cand_band is NULL), each one's squared deviation from
+// dense, and per head the eligible candidate with the least (the earlier on a tie).
+svga_status run_select(const void *q, const void *k, const void *v, const svga_problem *p,
+                       int n_cand, const int32_t *cand_type, const int32_t *cand_band,
+                       uint32_t eligible, const int32_t *w_spatial, const int32_t *w_temporal,
+                       const int32_t *rows, int n_rows, float scale, int32_t *type_out,
+                       int32_t *band_out, float *mse_out, int32_t *status_out, int device_out,
+                       void *ws, size_t ws_bytes, void *stream);
 svga_status run_classify(const void *q, const void *k, const void *v, const svga_problem *p,
                          const int32_t *w_spatial, const int32_t *w_temporal,
                          const int32_t *rows, int n_rows, float scale, int32_t *head_type_out,

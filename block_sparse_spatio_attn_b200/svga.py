@@ -35,7 +35,8 @@ EXPORTED = ["svga_problem_rows", "svga_block_map_size", "svga_build_block_map",
             "svga_validate_block_map", "svga_classify_heads_async", "svga_build_block_map_routed",
             "svga_permute_tokens_mapped", "svga_unpermute_tokens_mapped",
             "svga_dense_attention_fwd",
-            "svga_classify_size", "svga_classify_heads", "svga_last_error",
+            "svga_classify_size", "svga_classify_heads", "svga_kept_fraction",
+            "svga_autotune_size", "svga_autotune_heads", "svga_last_error",
             "svga_status_string", "svga_version"]
 
 
@@ -94,6 +95,10 @@ def load() -> ctypes.CDLL:
         lib.svga_classify_size.argtypes = [PP, I, ctypes.POINTER(SZ)]
         lib.svga_classify_heads.argtypes = [P, P, P, PP, P, P, P, I, F, P, P, P, SZ, P]
         lib.svga_classify_heads_async.argtypes = [P, P, P, PP, P, P, P, I, F, P, P, P, P, SZ, P]
+        lib.svga_kept_fraction.argtypes = [PP, I, I, ctypes.POINTER(ctypes.c_double)]
+        lib.svga_autotune_size.argtypes = [PP, I, I, ctypes.POINTER(SZ)]
+        lib.svga_autotune_heads.argtypes = [P, P, P, PP, P, P, I, ctypes.c_double, P, I, F, P,
+                                            P, P, P, SZ, P]
         lib.svga_build_block_map_routed.argtypes = [PP, P, P, P, ctypes.POINTER(BlockMapC), P,
                                                    SZ, P]
         lib.svga_permute_tokens_mapped.argtypes = [P, P, PP, ctypes.POINTER(BlockMapC), P]
@@ -396,6 +401,46 @@ def svga_classify_heads_async(q, k, v, problem: ProblemSpec, w_spatial, w_tempor
     _check(load().svga_classify_heads_async(
         pq, pk, pv, ctypes.byref(problem.c), wsp, wtp, pr, int(n_rows), float(scale), pt, pm,
         ps, _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def svga_kept_fraction(problem: ProblemSpec, head_type: int, band: int) -> float:
+    f = ctypes.c_double()
+    _check(load().svga_kept_fraction(ctypes.byref(problem.c), int(head_type), int(band),
+                                     ctypes.byref(f)))
+    return f.value
+
+
+def svga_autotune_size(problem: ProblemSpec, n_rows: int, n_cand: int) -> int:
+    sz = ctypes.c_size_t()
+    _check(load().svga_autotune_size(ctypes.byref(problem.c), int(n_rows), int(n_cand),
+                                     ctypes.byref(sz)))
+    return sz.value
+
+
+def svga_autotune_heads(q, k, v, problem: ProblemSpec, candidates, max_kept_fraction: float,
+                        rows, n_rows: int, scale: float, workspace=None, stream=None):
+    """candidates: [(type, band), ...].  Returns (types [heads], bands [heads],
+    mse [heads][n_cand])."""
+    a = _Args()
+    pq, pk, pv = a.tokens(problem, q=q, k=k, v=v)
+    pr = a.t(rows, "rows", torch.int32, numel=n_rows, optional=True)
+    n_cand = len(candidates)
+    need = svga_autotune_size(problem, n_rows, n_cand)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    pw = a.t(workspace, "workspace", torch.uint8)
+    a.done()
+    H = problem.heads
+    ct = (ctypes.c_int32 * n_cand)(*[int(c[0]) for c in candidates])
+    cb = (ctypes.c_int32 * n_cand)(*[int(c[1]) for c in candidates])
+    types = (ctypes.c_int32 * H)()
+    bands = (ctypes.c_int32 * H)()
+    mse = (ctypes.c_float * (H * n_cand))()
+    _check(load().svga_autotune_heads(pq, pk, pv, ctypes.byref(problem.c), ct, cb, n_cand,
+                                      float(max_kept_fraction), pr, int(n_rows), float(scale),
+                                      types, bands, mse, pw, workspace.numel(), _stream(stream)))
+    return (list(types), list(bands),
+            [list(mse[h * n_cand:(h + 1) * n_cand]) for h in range(H)])
 
 
 def svga_build_block_map_routed(problem: ProblemSpec, head_type_dev: torch.Tensor, w_spatial,

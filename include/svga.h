@@ -343,6 +343,48 @@ SVGA_API svga_status svga_classify_heads(const void *q, const void *k, const voi
                                 float scale, int32_t *head_type_out, float *mse_out, void *workspace,
                                 size_t workspace_bytes, svga_stream_t stream);
 
+/* ---- Band selection: the classifier over a list of candidate masks ----------------
+ * The pages choose between a spatial and a temporal mask per head by the least
+ * deviation from dense on a few query rows (aihirek.info, section "A Sparse VideoGen a
+ * figyelmi fejeket osztalyozza").  The calls below extend the choice to a list of
+ * candidate (type, band) masks.  The pages give no rule for trading a band's deviation
+ * against its cost (the least deviation alone always favours the widest band), so this
+ * library's reading is a budget: a candidate is eligible when the fraction of all
+ * (query, key) pairs its mask keeps is at most max_kept_fraction (the pages report
+ * about 39 % kept, aihirek.info, section "A TPU-kernel kialakitasa dontonek
+ * bizonyult"), and each head takes the eligible candidate whose output deviates least
+ * from dense (mean squared error over the sampled rows x head_dim), the earlier
+ * candidate on a tie. */
+
+/* Fraction of the N*N (query, key) pairs one head's mask keeps on this problem (the
+ * anchor included), counted exactly in closed form.  Host-only. */
+SVGA_API svga_status svga_kept_fraction(const svga_problem *problem, int head_type, int band,
+                                        double *fraction);
+
+/* Workspace for svga_autotune_heads with n_rows sampled rows and n_cand candidates
+ * (1 .. 16). */
+SVGA_API svga_status svga_autotune_size(const svga_problem *problem, int n_rows, int n_cand,
+                                        size_t *workspace_bytes);
+
+/* Per-head mask type and band among candidates.
+ *   q, k, v          : DEVICE bf16 [heads, tokens, head_dim], frame-major
+ *   cand_type/_band  : HOST int32 [n_cand]: SVGA_HEAD_SPATIAL / _TEMPORAL and 0..65535
+ *   max_kept_fraction: in (0, 1]; at least one candidate must keep no more than it
+ *                      (SVGA_ERR_INVALID_ARG otherwise)
+ *   rows, n_rows     : sampled query rows as for svga_classify_heads (NULL: the default
+ *                      rule)
+ *   head_type_out    : HOST int32 [heads];  band_out: HOST int32 [heads]
+ *   mse_out          : HOST float [heads][n_cand] or NULL: every candidate's deviation
+ *   workspace        : DEVICE, at least svga_autotune_size bytes, 256-byte aligned
+ * Synchronises `stream`.  The problem's head_type, band and order arrays are not read. */
+SVGA_API svga_status svga_autotune_heads(const void *q, const void *k, const void *v,
+                                         const svga_problem *problem, const int32_t *cand_type,
+                                         const int32_t *cand_band, int n_cand,
+                                         double max_kept_fraction, const int32_t *rows,
+                                         int n_rows, float scale, int32_t *head_type_out,
+                                         int32_t *band_out, float *mse_out, void *workspace,
+                                         size_t workspace_bytes, svga_stream_t stream);
+
 /* ---- Routed pipeline: the classifier's decision stays on the device -------------
  * The pages profile the heads online and then run the chosen sparse mask (aihirek.info,
  * section "A Sparse VideoGen a figyelmi fejeket osztalyozza").  The four calls below

@@ -274,3 +274,28 @@ def classify(q: np.ndarray, k: np.ndarray, v: np.ndarray, F: int, S: int, scale:
     ms = float(np.mean((os_ - od) ** 2))
     mt = float(np.mean((ot - od) ** 2))
     return (SPATIAL if ms <= mt else TEMPORAL), ms, mt
+
+
+def select_band(q: np.ndarray, k: np.ndarray, v: np.ndarray, F: int, S: int, scale: float,
+                candidates, anchor: int, rows: np.ndarray, max_kept_fraction: float):
+    """Per-head choice among candidate masks (type, band), extending the online profiling
+    the aihirek.info summary describes (section "A Sparse VideoGen a figyelmi fejeket
+    osztalyozza": keep the mask whose output deviates least from dense on a few query
+    rows) to several bands.  The pages give no cost rule, so a candidate is eligible when
+    its kept-pair fraction (counted pair by pair) is at most max_kept_fraction; among the
+    eligible ones the least mean squared deviation wins, the earlier on a tie.
+
+    Returns (index of the chosen candidate or -1, [mse per candidate],
+    [kept fraction per candidate])."""
+    N = F * S
+    od, _ = attention_rows(q, k, v, F, S, scale, DENSE, 0, anchor, rows)
+    mses, fracs = [], []
+    best = -1
+    for i, (t, w) in enumerate(candidates):
+        ox, _ = attention_rows(q, k, v, F, S, scale, t, w, anchor, rows)
+        mses.append(float(np.mean((ox - od) ** 2)))
+        fracs.append(kept_count(t, w, anchor, F, S) / float(N * N))
+        if fracs[-1] <= max_kept_fraction and (best < 0 or mses[-1] < mses[best]):
+            best = i
+    return best, mses, fracs
+

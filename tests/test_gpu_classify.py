@@ -79,3 +79,64 @@ def test_classify_2k_one_percent():
                                           wl.cand_temporal, None, n, 1.0 / math.sqrt(128))
     assert types == [0] * 5 + [1] * 5
     assert all(m[0] > 0 and m[1] > 0 for m in mse)
+
+
+def check_autotune(wl, q, k, v, n_rows, cands, budget, heads=None):
+    """GPU band selection against oracle.select_band on the same rows: every eligible
+    candidate's deviation within 2e-2 relative, and the same choice unless the two best
+    eligible deviations lie within 1e-2 of each other."""
+    prob = svga.ProblemSpec.from_workload(wl)
+    rows = default_sample_rows(wl.tokens, n_rows)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    types, bands, mse = svga.svga_autotune_heads(q.cuda(), k.cuda(), v.cuda(), prob, cands,
+                                                 budget, None, n_rows, scale)
+    F, S = wl.frames, wl.tokens_per_frame
+    for h in (range(wl.heads) if heads is None else heads):
+        best, mses, fracs = oracle.select_band(q[h].float().numpy(), k[h].float().numpy(),
+                                               v[h].float().numpy(), F, S, scale, cands,
+                                               wl.anchor_frame0, rows.numpy(), budget)
+        for c, (g, m) in enumerate(zip(mse[h], mses)):
+            assert abs(g - m) <= MSE_REL * m, (h, c, g, m)
+        elig = sorted(m for m, f in zip(mses, fracs) if f <= budget)
+        if len(elig) < 2 or elig[1] - elig[0] > TIE_REL * elig[1]:
+            assert (types[h], bands[h]) == tuple(cands[best]), (h, types[h], bands[h], best)
+    return types, bands
+
+
+def test_autotune_small_against_oracle():
+    wl = C.Workload("struct_small", 7, 6, 10, 64, [0, 0, 1, 1], [1, 1, 40, 40], [0] * 4,
+                    seed=4, structured=True)
+    q, k, v = make_qkv(wl)
+    cands = [(0, 0), (0, 1), (0, 2), (1, 10), (1, 20), (1, 40)]
+    types, bands = check_autotune(wl, q, k, v, 60, cands, 0.6)
+    assert types == [0, 0, 1, 1]
+
+
+def test_autotune_budget_excludes_wide_bands():
+    """A budget that only the narrow candidates meet: no head takes a wider one."""
+    wl = C.Workload("struct_small", 7, 6, 10, 64, [0, 0, 1, 1], [1, 1, 40, 40], [0] * 4,
+                    seed=4, structured=True)
+    q, k, v = make_qkv(wl)
+    prob = svga.ProblemSpec.from_workload(wl)
+    cands = [(0, 0), (0, 3), (1, 5), (1, 40)]
+    fr = [svga.svga_kept_fraction(prob, t, b) for t, b in cands]
+    budget = max(fr[0], fr[2]) + 1e-9
+    assert fr[1] > budget and fr[3] > budget
+    types, bands = check_autotune(wl, q, k, v, 60, cands, budget)
+    assert all((t, b) in ((0, 0), (1, 5)) for t, b in zip(types, bands))
+    with pytest.raises(svga.SvgaError):   # nothing eligible
+        svga.svga_autotune_heads(q.cuda(), k.cuda(), v.cuda(), prob, cands, min(fr) / 2, None,
+                                 60, 0.125)
+
+
+def test_autotune_2k_structured():
+    """2K structured inputs, bands around the classifier's candidates under the pages'
+    kept budget (38.87 %): frame-local heads pick a spatial band, same-position heads a
+    temporal one; heads 0 and 9 checked against the oracle on 48 rows."""
+    wl = C.twok()
+    q, k, v = make_qkv(wl)
+    cands = [(0, 2), (0, 3), (0, 4), (1, 1200), (1, 2400), (1, 4800)]
+    types, bands = check_autotune(wl, q, k, v, 48, cands, 0.3887, heads=(0, 9))
+    assert types == [0] * 5 + [1] * 5
+    assert all(b in (2, 3) for b in bands[:5]) and all(b in (1200, 2400) for b in bands[5:])
+
