@@ -274,6 +274,7 @@ def run_svga(args, rank, world, local_rank):
 
     qp, kp, vp, op, o = (torch.empty_like(qd) for _ in range(5))
 
+    kernel_flag = svga.FLAG_CTA_PAIR if args.cta_pair else 0
     # One step: K and V move to each head's token order; the attention kernel gathers
     # the Q rows from frame-major memory itself and writes O rows back frame-major.
     def step(attn_evs=None):
@@ -282,7 +283,8 @@ def run_svga(args, rank, world, local_rank):
         if attn_evs is not None:
             attn_evs[0].record(stream)
         svga.svga_sparse_attention_fwd_part(qd, kp, vp, o, None, prob, bmap, scale,
-                                            svga.FLAG_QO_FRAME_MAJOR, part, n_parts)
+                                            svga.FLAG_QO_FRAME_MAJOR | kernel_flag, part,
+                                            n_parts)
         if attn_evs is not None:
             attn_evs[1].record(stream)
 
@@ -293,7 +295,7 @@ def run_svga(args, rank, world, local_rank):
         svga.svga_sparse_attention_fwd(qp, kp, vp, op, None, prob, bmap, scale)
         svga.svga_unpermute_tokens(op, o, prob)
 
-    launches_per_step = 3
+    launches_per_step = 4 if args.cta_pair else 3  # the pair kernel, then the rest
     if args.mode == "parts":
         # study of one problem split over P GPUs: each part timed alone on this GPU,
         # which is the whole of what one of P GPUs would run (no exchange between parts)
@@ -328,7 +330,7 @@ def run_svga(args, rank, world, local_rank):
         step_separate()
         for _ in range(args.warmup + args.steps):   # the launch the timed step makes
             svga.svga_sparse_attention_fwd(qd, kp, vp, o, None, prob, bmap, scale,
-                                           svga.FLAG_QO_FRAME_MAJOR)
+                                           svga.FLAG_QO_FRAME_MAJOR | kernel_flag)
         torch.cuda.synchronize()
         if bmap.device_status() != 0:
             raise RuntimeError(f"device status {bmap.device_status()}")
@@ -527,6 +529,7 @@ def run_svga(args, rank, world, local_rank):
                    "frames": wl.frames, "grid": f"{wl.grid_h}x{wl.grid_w}",
                    "head_types": "".join("ST"[t] for t in wl.head_type), "bands": wl.band,
                    "orders": wl.order, "tile": f"{wl.tile_q}x{wl.tile_k}",
+                   "attention_kernel": "cta_pair" if args.cta_pair else "one_cta",
                    "parallelism": (f"parts{world}" if split else f"replicas{world}")
                    if world > 1 else "single",
                    "l2": "inputs larger than L2 (Q,K,V %.0f MB)" % (3 * H * N * d * 2 / 1e6),
@@ -653,6 +656,8 @@ def main():
     ap.add_argument("--split", action="store_true",
                     help="under torchrun, the ranks share one problem (each runs its part of "
                          "the work items) instead of running one problem each")
+    ap.add_argument("--cta-pair", action="store_true",
+                    help="run the work items on CTA pairs (SVGA_FLAG_CTA_PAIR)")
     ap.add_argument("--mode", default="full", choices=["full", "attn", "parts", "classify"],
                     help="attn: only launch the attention kernel (for ncu captures)")
     args = ap.parse_args()

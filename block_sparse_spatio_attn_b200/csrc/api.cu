@@ -411,7 +411,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     }
     if ((rc = check_map_plan(g, map)) != SVGA_OK) return rc;
     if (flags & ~(SVGA_FLAG_NAIVE_B1 | SVGA_FLAG_TILE_ALIGNED | SVGA_FLAG_TEST_STALL |
-                  SVGA_FLAG_QO_FRAME_MAJOR | SVGA_FLAG_KV_FRAME_MAJOR)) {
+                  SVGA_FLAG_QO_FRAME_MAJOR | SVGA_FLAG_KV_FRAME_MAJOR | SVGA_FLAG_CTA_PAIR)) {
         set_error("unknown flags 0x%x", flags);
         return SVGA_ERR_INVALID_ARG;
     }
@@ -462,6 +462,7 @@ svga_status sparse_fwd_common(const void *q, const void *k, const void *v, void 
     a.test_stall = (flags & SVGA_FLAG_TEST_STALL) ? 1 : 0;
     a.qo_fm = (flags & SVGA_FLAG_QO_FRAME_MAJOR) ? 1 : 0;
     a.kv_fm = (flags & SVGA_FLAG_KV_FRAME_MAJOR) ? 1 : 0;
+    a.cta_pair = (flags & SVGA_FLAG_CTA_PAIR) ? 1 : 0;
     a.kn = g.kn;
     a.tile_q = g.tile_q;
     a.tile_k = g.tile_k;

@@ -104,6 +104,8 @@ struct KParams {
     int ksplit;
     float *part_o;
     float2 *part_ml;
+    // plan mode after the pair kernel: run only the items the pair kernel leaves
+    int pair_rest;
 };
 
 template <int D, int KN>
@@ -171,17 +173,24 @@ struct Item {
 // num_parts consecutive items, part r takes item r when g is even and num_parts-1-r when
 // g is odd, which keeps the parts' total work within one item of each other.  Under a
 // key-range split the ksplit consecutive CTAs of one item share its g.
+__device__ __forceinline__ int plan_item_of_slot(const KParams &p, int g)
+{
+    const int r = p.part, n = p.num_parts;
+    return g * n + ((g & 1) ? n - 1 - r : r);
+}
+
+// The CTAs of one work item: ksplit key-range parts, or the two CTAs of a pair.
+__device__ __forceinline__ int item_slot(const KParams &p) { return blockIdx.x / p.ksplit; }
 __device__ __forceinline__ int plan_item_of_block(const KParams &p)
 {
-    const int g = blockIdx.x / p.ksplit, r = p.part, n = p.num_parts;
-    return g * n + ((g & 1) ? n - 1 - r : r);
+    return plan_item_of_slot(p, item_slot(p));
 }
 
 // A caller's plan must describe this launch before any of its offsets is used: the
 // header against the launch's shape, tiles, anchor and item count, then this CTA's work
 // item (head, even first block, entry range inside the plan) and the head's info.
 // Every thread of the CTA reads the same words, so the verdict is uniform.
-__device__ __forceinline__ bool plan_matches(const KParams &p, int kn)
+__device__ __forceinline__ bool plan_matches(const KParams &p, int kn, int slot)
 {
     const int4 *h4 = reinterpret_cast<const int4 *>(p.hdr);
     // {magic, heads, tokens, frames}, {tokens_per_frame, anchor, tile_q, tile_k},
@@ -193,7 +202,7 @@ __device__ __forceinline__ bool plan_matches(const KParams &p, int kn)
           c.y == p.n_qblk && c.z == p.n_kc && c.w == p.n_items && d.z == p.Sp &&
           p.nq_rows == p.F * p.Sp && p.nk_rows == p.nq_rows))
         return false;
-    const int4 x = __ldg(p.items + plan_item_of_block(p));
+    const int4 x = __ldg(p.items + plan_item_of_slot(p, slot));
     if (!(x.x >= 0 && x.x < p.heads && x.y >= 0 && !(x.y & 1) && x.y < p.n_qblk && x.z >= 0 &&
           x.w >= 0 && x.w <= p.n_kc && (long long)x.z + x.w <= entry_cap))
         return false;
@@ -202,7 +211,7 @@ __device__ __forceinline__ bool plan_matches(const KParams &p, int kn)
            hi.z <= ORDER_TM_STRICT;
 }
 
-__device__ __forceinline__ Item make_item(const KParams &p, int kn)
+__device__ __forceinline__ Item make_item(const KParams &p, int kn, int slot, int kpart)
 {
     Item it;
     it.mode = p.mode;
@@ -211,20 +220,20 @@ __device__ __forceinline__ Item make_item(const KParams &p, int kn)
     it.ragged = (p.nk_rows % kn) != 0;
     int e_all;  // entries of the whole item
     if (p.mode == 0) {
-        const int4 x = __ldg(p.items + plan_item_of_block(p));
+        const int4 x = __ldg(p.items + plan_item_of_slot(p, slot));
         it.h = x.x;
         it.b0 = x.y;
         it.ent = p.entries + x.z;
         e_all = x.w;
     } else {
-        const int item = blockIdx.x / p.ksplit;
+        const int item = slot;
         it.h = item / p.n_pairs;
         it.b0 = 2 * (item - it.h * p.n_pairs);
         it.ent = nullptr;
         e_all = p.n_kc;
     }
     // this CTA's share of the entries (all of them without a key-range split)
-    const int r = blockIdx.x % p.ksplit;
+    const int r = kpart;
     const int e0 = (int)((long long)r * e_all / p.ksplit);
     const int e1 = (int)((long long)(r + 1) * e_all / p.ksplit);
     if (it.ent) it.ent += e0;
@@ -232,6 +241,20 @@ __device__ __forceinline__ Item make_item(const KParams &p, int kn)
     it.E = e1 - e0;
     it.valid1 = it.b0 + 1 < p.n_qblk;
     return it;
+}
+
+// Does the CTA pair run this item?  It takes items whose two 128-row blocks both exist
+// and both visit at least one key chunk; the rest (the last item of a head with an odd
+// number of blocks, items one of whose blocks visits nothing) run in the one-CTA kernel.
+// Every thread of the CTA calls it; the entries are scanned by all threads together.
+__device__ __forceinline__ bool item_fits_pair(const Item &it)
+{
+    if (!it.valid1) return false;
+    uint32_t any = 0u;
+    for (int n = threadIdx.x; n < it.E; n += blockDim.x) any |= it.raw(n);
+    const int has0 = __syncthreads_or((int)(any & kEntV0));
+    const int has1 = __syncthreads_or((int)(any & kEntV1));
+    return has0 && has1;
 }
 
 // Set bits [c0, c1) of a mask of NW 32-bit words (0 <= c0 < c1 <= 32 * NW).
@@ -368,12 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.mode == 0 && plan_item_of_block(p) >= p.n_items) return;  // the last group ran out
-    if (p.mode == 0 && p.check_plan && !plan_matches(p, KN)) {
+    if (p.mode == 0 && p.check_plan && !plan_matches(p, KN, item_slot(p))) {
         // a map built for another problem: report it and touch nothing
         if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int32_t)SVGA_ERR_INVALID_ARG);
         return;
     }
-    const Item it = make_item(p, KN);
+    const Item it = make_item(p, KN, item_slot(p), blockIdx.x % p.ksplit);
+    if (p.pair_rest && item_fits_pair(it)) return;  // the pair kernel ran this item
     // keys of a head in a temporal-major order, read from frame-major K and V: warps 0 and
     // 2 gather the chunk rows instead of the TMA producer's tile loads
     const bool kv_gather = p.kv_fm && p.mode == 0 && __ldg(p.head_info + it.h).z != ORDER_FM;
@@ -448,8 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issued = idx + 1;
                 }
             }
-            if (!ok) {
-                // Abort: let the copies in flight land before the CTA exits.
+            {
+                // Every copy this thread issued lands before the CTA can exit, whichever
+                // role aborts (in a normal run they have all landed already).
                 if (q_tma) mbar_wait_bounded(qf, 0);
                 for (int idx = (issued > C::kStages ? issued - C::kStages : 0); idx < issued; ++idx)
                     if (!(p.test_stall && idx == 0))
@@ -943,6 +968,522 @@ EncodeTiledFn get_encode_fn()
 }
 
 // [heads, rows, d] bf16, box = 64 columns x box_rows rows x 1 head, 128-byte swizzle.
+// ============================================================================
+// The pair kernel (SVGA_FLAG_CTA_PAIR): a work item (two 128-row query blocks) runs on a
+// CTA pair over two SMs.  Each tcgen05.mma covers M = 256 rows (both blocks); CTA r
+// holds block r's Q rows, S and O, and half of every K chunk (keys r*64 .. r*64+63) and
+// of every V chunk (head-dim columns r*64 .. r*64+63), so each SM loads half the K/V
+// bytes the one-CTA kernel loads per item.  The TMEM this frees (one block per CTA)
+// holds two S tiles, so the S of a visit is computed while the softmax works on the
+// previous one.
+//   * TMEM per CTA: S0 | S1 (128 columns each) | P0 | P1 (64 each, bf16 pairs) | O (128);
+//     visit k uses S and P buffer k % 2;
+//   * warp 0: TMA producer (own Q rows, own halves of K / V) into 16 KB stages; a
+//     stage's copies complete on this CTA's barrier;
+//   * rank 0: warp 1 issues the S products, warp 2 the P V products (the issuing warps
+//     slow the softmax warps that share their SM sub-partition, so they sit on two
+//     different ones).  Rank 1, warp 1: forwards its Q and stage completions to rank 0
+//     (one remote arrival each);
+//   * warps 4-7 and 8-11: two softmax groups of whole rows (TMEM lane = row); group g
+//     takes the visits k with k % 2 == g, and the groups pass each row's reference
+//     maximum from visit to visit;
+//   * every wait is bounded; an abort stops every role of the CTA, drains its copies
+//     and (rank 0) its MMAs, and the pair meets at a cluster barrier before TMEM is
+//     released.
+// Arrivals on the peer's barriers use the default (CTA-scope) release: what they hand
+// over is tensor memory the caller completed and fenced, or copies complete on the
+// caller's own barrier.  A cluster-scope release there cost a memory barrier per
+// hand-off and made the kernel 40 % slower.
+namespace pair {
+
+constexpr int kThreads = 384;
+constexpr int kD = 128, kKN = 128;
+constexpr int kQBytes = 128 * kD * 2;        // the CTA's 128 Q rows
+constexpr int kQChunk = 128 * 64 * 2;         // one 64-column half of the Q rows
+constexpr int kStageBytes = 16384;            // a K half (64 keys x 128) or V half (128 x 64)
+constexpr int kKHalfChunk = 64 * 64 * 2;      // 64 keys x 64 columns of a K half
+constexpr int kStages = 10;
+constexpr uint32_t kPS = 0, kPP = 256, kPO = 384;  // TMEM columns: S0|S1, P0|P1, O
+constexpr int kRows = 128;                    // rows of the CTA's block
+constexpr float kRaiseLog2 = 8.f;             // a tile this far above the reference raises it
+
+struct Bars {
+    uint64_t q_full;              // own Q rows landed (TMA bytes, or the gather's arrival)
+    uint64_t peer_q;              // rank 0: rank 1's Q landed
+    uint64_t kv_full[kStages];    // own half of the stage landed
+    uint64_t peer_full[kStages];  // rank 0: rank 1's half landed
+    uint64_t kv_empty[kStages];   // the MMAs reading the stage are done (both CTAs)
+    uint64_t s_full[2];           // S buffer b computed (both CTAs)
+    uint64_t s_free[2];           // rank 0: S buffer b read by its group's 8 warps (2 CTAs)
+    uint64_t p_full[2];           // rank 0: P buffer b written by its group's 8 warps
+    uint64_t o_done[2];           // the P V reading P buffer b is done (both CTAs)
+    uint64_t o_final;             // every P V of the item is done (both CTAs)
+    uint64_t ref_bar[2];          // the reference after visit k (k % 2 = b) is in m_ref
+    uint64_t p_local[2];          // this CTA's group wrote P buffer b
+    uint64_t fin_bar;             // both groups' sums are in fin_m / fin_l
+    uint64_t drain[2];            // rank 0's issuers, after an abort
+    uint32_t tmem_base;
+    int abort;
+    float m_ref[kRows];           // each row's reference maximum (exp2 domain)
+    float fin_m[2][kRows];        // per group: the reference of its sum
+    float fin_l[2][kRows];        // per group: its sum of P
+};
+constexpr int kSmemData = kQBytes + kStages * kStageBytes;
+constexpr int kSmemLaunch = kSmemData + (int)sizeof(Bars) + 1024;
+
+}  // namespace pair
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
+    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK64,
+                         const __grid_constant__ CUtensorMap tmV, const KParams p)
+{
+    using namespace pair;
+    constexpr int D = kD, KN = kKN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sKV = smem + kQBytes;
+    Bars *bar = reinterpret_cast<Bars *>(smem + kSmemData);
+    volatile int *abort_flag = &bar->abort;
+
+    const uint32_t rank = cluster_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = blockIdx.x >> 1;
+    // both CTAs of the pair take the same decisions here: same item, same plan
+    if (plan_item_of_slot(p, slot) >= p.n_items) return;  // the last group ran out
+    if (p.check_plan && !plan_matches(p, KN, slot)) {
+        if (threadIdx.x == 0 && rank == 0 && p.status)
+            atomicCAS(p.status, 0, (int32_t)SVGA_ERR_INVALID_ARG);
+        return;
+    }
+    const Item it = make_item(p, KN, slot, 0);
+    if (!item_fits_pair(it)) return;  // both CTAs decide alike: the one-CTA kernel runs it
+    const int4 hinfo = __ldg(p.head_info + it.h);
+    const bool q_tma = !p.qo_fm || hinfo.z == ORDER_FM;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar->q_full), 1);
+        mbar_init(smem_u32(&bar->peer_q), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&bar->kv_full[s]), 1);
+            mbar_init(smem_u32(&bar->peer_full[s]), 1);
+            mbar_init(smem_u32(&bar->kv_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bar->s_full[b]), 1);
+            mbar_init(smem_u32(&bar->s_free[b]), 8);
+            mbar_init(smem_u32(&bar->p_full[b]), 8);
+            mbar_init(smem_u32(&bar->ref_bar[b]), 4);
+            mbar_init(smem_u32(&bar->p_local[b]), 4);
+            mbar_init(smem_u32(&bar->o_done[b]), 1);
+            mbar_init(smem_u32(&bar->drain[b]), 1);
+        }
+        mbar_init(smem_u32(&bar->o_final), 1);
+        mbar_init(smem_u32(&bar->fin_bar), 8);
+        bar->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&bar->tmem_base), 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+    const int total = 2 * it.E;  // stages: K then V of each entry
+    const int blk = it.b0 + (int)rank;
+
+    if (warp < 4) {
+        setmaxnreg_dec<kRegsLow>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- TMA producer
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK64);
+            prefetch_tmap(&tmV);
+            const uint32_t qf = smem_u32(&bar->q_full);
+            if (q_tma) {
+                // a block past the last one reads zeros (the box is out of range)
+                mbar_arrive_expect_tx(qf, kQBytes);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(smem_u32(sQ + c * kQChunk), &tmQ, qf, 64 * c, blk * kBlockM, it.h);
+            }
+            int issued = 0;
+            bool ok = true;
+            uint32_t e_nxt = it.E > 0 ? it.raw(0) : 0u;
+            for (int n = 0; n < it.E && ok; ++n) {
+                const int kc = (int)(e_nxt & kEntChunkMask);
+                e_nxt = it.raw(min(n + 1, it.E - 1));
+                for (int t = 0; t < 2; ++t) {
+                    const int idx = 2 * n + t, s = idx % kStages, round = idx / kStages;
+                    if (round > 0 &&
+                        !mbar_wait(smem_u32(&bar->kv_empty[s]), (round - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (p.test_stall && idx == 0) {  // nothing ever completes this stage
+                        issued = idx + 1;
+                        continue;
+                    }
+                    const uint32_t fb = smem_u32(&bar->kv_full[s]);
+                    const uint32_t dst = smem_u32(sKV + s * kStageBytes);
+                    const int krow = kc * KN + (int)rank * 64;
+                    if (t == 0 && krow >= p.nk_rows) {
+                        // This half of the last chunk holds no key: no copy is issued, the
+                        // stage keeps stale rows, and every key of it is masked (the last
+                        // chunk is never a full one), so its P is zero; its V rows are
+                        // zeros, read by a box that starts inside the tensor.
+                        mbar_arrive(fb);
+                    } else if (t == 0) {  // keys kc*128 + rank*64 .. +63, both column halves
+                        mbar_arrive_expect_tx(fb, kStageBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            tma_load_3d(dst + c * kKHalfChunk, &tmK64, fb, 64 * c, krow, it.h);
+                    } else {  // all 128 keys, columns rank*64 .. +63
+                        mbar_arrive_expect_tx(fb, kStageBytes);
+                        tma_load_3d(dst, &tmV, fb, 64 * (int)rank, kc * KN, it.h);
+                    }
+                    issued = idx + 1;
+                }
+            }
+            {  // every copy issued lands before the CTA can exit, whichever role aborts
+                if (q_tma) mbar_wait_bounded(qf, 0);
+                for (int idx = (issued > kStages ? issued - kStages : 0); idx < issued; ++idx)
+                    if (!(p.test_stall && idx == 0))
+                        mbar_wait_bounded(smem_u32(&bar->kv_full[idx % kStages]),
+                                          (idx / kStages) & 1);
+            }
+        } else if (warp == 1 && lane == 0 && rank == 1) {
+            // ------------------------------------ rank 1: completions to rank 0
+            const uint32_t peer_q = cluster_addr(smem_u32(&bar->peer_q), 0);
+            if (mbar_wait(smem_u32(&bar->q_full), 0, abort_flag)) {
+                mbar_arrive_cluster(peer_q);
+                for (int idx = 0; idx < total; ++idx) {
+                    const int s = idx % kStages;
+                    if (!mbar_wait(smem_u32(&bar->kv_full[s]), (idx / kStages) & 1, abort_flag))
+                        break;
+                    mbar_arrive_cluster(cluster_addr(smem_u32(&bar->peer_full[s]), 0));
+                }
+            }
+        } else if ((warp == 1 || warp == 2) && lane == 0 && rank == 0) {
+            // ------------------------------------------------ rank 0: MMA issuers
+            const bool s_role = warp == 1;
+            constexpr uint32_t idS = idesc_bf16_f32(256, KN, 0);
+            constexpr uint32_t idO = idesc_bf16_f32(256, D, 1);
+            const uint64_t dK = smem_desc_sw128(0, 16, 1024);
+            const uint64_t dV = smem_desc_sw128(0, 16, 1024);
+            const uint32_t q_addr = smem_u32(sQ) >> 4, kv_addr = smem_u32(sKV) >> 4;
+            bool ok = true;
+            if (s_role)
+                ok = mbar_wait(smem_u32(&bar->q_full), 0, abort_flag) &&
+                     mbar_wait(smem_u32(&bar->peer_q), 0, abort_flag);
+            tc_fence_after();
+            // both halves of stage idx are in place
+            auto wait_full = [&](int idx) {
+                const int s = idx % kStages;
+                const uint32_t ph = (idx / kStages) & 1;
+                return mbar_wait(smem_u32(&bar->kv_full[s]), ph, abort_flag) &&
+                       mbar_wait(smem_u32(&bar->peer_full[s]), ph, abort_flag);
+            };
+            auto release = [&](int idx) {
+                if (idx + kStages < total) mma_commit_pair(smem_u32(&bar->kv_empty[idx % kStages]));
+            };
+            for (int k = 0; k < it.E && ok; ++k) {
+                const int b = k & 1;
+                if (s_role) {
+                    // S of visit k into S buffer b, once visit k-2's S was read there
+                    if (k >= 2 &&
+                        !(ok = mbar_wait(smem_u32(&bar->s_free[b]), ((k >> 1) - 1) & 1, abort_flag)))
+                        break;
+                    if (!(ok = wait_full(2 * k))) break;
+                    tc_fence_after();
+                    const uint64_t a0 = dK + q_addr;
+                    const uint64_t b0 = dK + (kv_addr + ((2 * k) % kStages) * (kStageBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss_pair(tmem + kPS + b * 128,
+                                    a0 + (uint32_t)(((kk >> 2) * kQChunk + (kk & 3) * 32) >> 4),
+                                    b0 + (uint32_t)(((kk >> 2) * kKHalfChunk + (kk & 3) * 32) >> 4),
+                                    idS, kk > 0 ? 1u : 0u);
+                    mma_commit_pair(smem_u32(&bar->s_full[b]));
+                    release(2 * k);
+                } else {
+                    // O += P V of visit k, once both CTAs wrote P buffer b
+                    if (!(ok = mbar_wait(smem_u32(&bar->p_full[b]), (k >> 1) & 1, abort_flag)))
+                        break;
+                    if (!(ok = wait_full(2 * k + 1))) break;
+                    tc_fence_after();
+                    const uint64_t b0 =
+                        dV + (kv_addr + ((2 * k + 1) % kStages) * (kStageBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < KN / 16; ++kk)
+                        mma_ts_pair(tmem + kPO, tmem + kPP + b * 64 + kk * 8,
+                                    b0 + (uint32_t)((kk * 2048) >> 4), idO,
+                                    (k > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit_pair(smem_u32(&bar->o_done[b]));
+                    release(2 * k + 1);
+                }
+            }
+            // the epilogue's signal: every P V of the item is done
+            if (ok && !s_role && it.E > 0) mma_commit_pair(smem_u32(&bar->o_final));
+            if (!ok) {  // every MMA this thread issued is done before TMEM is released
+                const uint32_t drain = smem_u32(s_role ? &bar->drain[0] : &bar->drain[1]);
+                mma_commit_pair_self(drain);
+                mbar_wait_bounded(drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------ softmax groups
+        // Group g (warps 4-7 or 8-11) takes the visits k with k % 2 == g, whole rows
+        // (thread = TMEM lane = row of this CTA's block).  The groups run half a visit
+        // apart, so the exponentials of one overlap the waits of the other.  They share
+        // each row's reference maximum: the group of visit k reads the reference visit
+        // k-1 left, raises it when the tile's maximum lies more than kRaiseLog2 above it
+        // (the row's first kept keys set it), and passes it on.  Every P is then at most
+        // 2^kRaiseLog2.  Each group keeps its own running sum; the epilogue adds them.
+        setmaxnreg_inc<kRegsHigh>();
+        const int g = (warp - 4) >> 2, quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const uint32_t tO = tmem + lane_base + kPO;
+        const int qpos = blk * kBlockM + row;
+        const bool row_valid = qpos < p.nq_rows;
+        const int type = hinfo.x, band = hinfo.y, korder = hinfo.z;
+        int fq = 0, sq = 0;
+        bool q_tok = row_valid;  // false: a position of the padded layout without a token
+        if (row_valid) {
+            if (korder == ORDER_FM) {
+                fq = qpos / p.Sp;
+                sq = qpos - fq * p.Sp;
+                q_tok = sq < p.S;
+            } else {
+                q_tok = qpos < p.N;
+                if (q_tok) pos_to_coord(korder, qpos, p.F, p.S, fq, sq);
+            }
+        }
+        int tok = qpos;
+        if (p.qo_fm && row_valid) tok = fq * p.S + sq;
+        if (!q_tma) {
+            // Q rows gathered from their frame-major tokens: group g copies head-dim
+            // columns g*64 .. g*64+63 of its row into the swizzled Q tile
+            const uint32_t qs = smem_u32(sQ + g * kQChunk) + row * 128;
+            const uint4 *src = static_cast<const uint4 *>(p.q) +
+                               ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * (D / 8) + g * 8;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint4 x = row_valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+                st_shared_v4(qs + ((u ^ (row & 7)) << 4), x.x, x.y, x.z, x.w);
+            }
+            fence_proxy_async_smem();  // generic-proxy stores -> visible to the MMA
+            named_bar_sync(1, 256);    // every row of the tile is in place
+            if (warp == 4 && lane == 0) mbar_arrive(smem_u32(&bar->q_full));
+        }
+        const uint32_t vbit = rank ? kEntV1 : kEntV0, fbit = rank ? kEntF1 : kEntF0;
+        const uint32_t s_free0 = cluster_addr(smem_u32(&bar->s_free[0]), 0);
+        const uint32_t p_full0 = cluster_addr(smem_u32(&bar->p_full[0]), 0);
+        const float sl2 = p.scale_log2;
+        float m_seen = -INFINITY, l = 0.f;  // this group's sum, in units of 2^m_seen
+        bool ok = true;
+        // all lanes wait (bounded) for a phase; tensor-memory reads may follow
+        auto wait_all = [&](uint32_t b_addr, uint32_t parity) {
+            const bool w = __all_sync(0xffffffffu, mbar_wait(b_addr, parity, abort_flag));
+            tc_fence_after();
+            return w;
+        };
+        uint32_t r[KN];
+        auto tile_max = [&]() {
+            float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < KN; c += 8) {
+                a0 = fmax3(a0, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+                a1 = fmax3(a1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+                a2 = fmax3(a2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+                a3 = fmax3(a3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+            }
+            return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+        };
+        uint32_t e_next = g < it.E ? it.raw(g) : 0u;  // prefetched, fixed where used
+        for (int k = g; k < it.E; k += 2) {
+            const int b = k & 1;  // this group's S and P buffers
+            const uint32_t e = it.fix(e_next);
+            e_next = it.raw(min(k + 2, it.E - 1));
+            const bool visits = (e & vbit) != 0;  // the same for the whole CTA
+            if (!(ok = wait_all(smem_u32(&bar->s_full[b]), (k >> 1) & 1))) break;
+            const int kc = (int)(e & kEntChunkMask);
+            const bool full = p.aligned ? (kc + 1) * KN <= p.nk_rows : (e & fbit) != 0;
+            uint32_t keep[KN / 32];
+            if (visits) {
+                const uint32_t tS = tmem + lane_base + kPS + b * 128;
+#pragma unroll
+                for (int j = 0; j < KN / 32; ++j)
+                    tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[j * 32]));
+                if (!full)  // mask computed while the TMEM load is in flight
+                    keep_mask<KN>(korder, p.aligned ? MASK_DENSE : type, band, p.anchor, p.F,
+                                  p.S, p.Sp, korder == ORDER_FM ? p.nk_rows : p.N, q_tok, fq,
+                                  sq, kc * KN, keep);
+                tmem_wait_ld();
+            }
+            // S is in registers: S buffer b may take visit k+2's S
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(s_free0 + b * 8);
+            if (visits && !full) {
+#pragma unroll
+                for (int c = 0; c < KN; ++c)
+                    if (!((keep[c >> 5] >> (c & 31)) & 1u)) r[c] = kNegInfBits;
+            }
+            float m_cur = -INFINITY;  // the reference visit k-1 left
+            if (k >= 1) {
+                if (!(ok = wait_all(smem_u32(&bar->ref_bar[b ^ 1]), ((k - 1) >> 1) & 1))) break;
+                m_cur = bar->m_ref[row];
+            }
+            if (m_cur != m_seen) {  // raised by the other group: this group's sum follows
+                l *= fast_exp2(m_seen - m_cur);
+                m_seen = m_cur;
+            }
+            float m_new = m_cur;
+            if (visits) {
+                const float t = tile_max();
+                if (t > m_cur + kRaiseLog2) m_new = t;
+            }
+            // A raised reference rescales O, which holds the P V of visits up to k-1 in
+            // units of 2^m_cur, once the last of them is done.  A row whose reference is
+            // set for the first time has a zero O row and needs none.  (Rare.)  A warp
+            // that raises first waits for the other group's P of visit k-1, which that
+            // group wrote after it saw the P V of visit k-3 done; and it passes the
+            // reference on only then, so that group cannot write the P of visit k+1 in
+            // the meantime.  Both barriers waited for here are thus one phase from the
+            // phase they are at.
+            const bool raise = m_new > m_cur && m_cur != -INFINITY;
+            const bool any_raise = __any_sync(0xffffffffu, raise);
+            if (any_raise &&
+                !(ok = wait_all(smem_u32(&bar->p_local[b ^ 1]), ((k - 1) >> 1) & 1)))
+                break;
+            bar->m_ref[row] = m_new;
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar->ref_bar[b]));
+            if (any_raise) {
+                if (!(ok = wait_all(smem_u32(&bar->o_done[b ^ 1]), ((k - 1) >> 1) & 1))) break;
+                const float fac = raise ? fast_exp2(m_cur - m_new) : 1.f;
+#pragma unroll 1
+                for (int j = 0; j < D / 32; ++j) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + j * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fac);
+                    tmem_st32(tO + j * 32, o);
+                }
+                tmem_wait_st();
+            }
+            if (m_new != m_seen) {
+                l *= fast_exp2(m_seen - m_new);
+                m_seen = m_new;
+            }
+            // P buffer b: the P V of visit k-2 read it
+            if (k >= 2 && !(ok = wait_all(smem_u32(&bar->o_done[b]), ((k - 2) >> 1) & 1))) break;
+            const uint32_t tP = tmem + lane_base + kPP + b * 64;
+            if (!visits) {  // the other block's chunk: this block adds nothing
+                uint32_t z[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) z[c] = 0u;
+                tmem_st32(tP, z);
+                tmem_st32(tP + 32, z);
+            } else {
+                // P = 2^(x sl2 - m_new) of every column, packed to bf16 into P buffer b
+                const float ms = (m_new == -INFINITY) ? 0.f : m_new;
+                const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ms, -ms);
+                float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < KN / 32; ++j) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const int c = j * 32 + 2 * c2;
+                        const float2 x = ffma2(
+                            make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2, nm2);
+                        const float2 ev = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                        if (c2 & 1)
+                            s1 = fadd2(s1, ev);
+                        else
+                            s0 = fadd2(s0, ev);
+                        pk[c2] = pack_bf16x2_int(ev.x, ev.y);
+                    }
+                    tmem_st16(tP + j * 16, pk);
+                }
+                l += (s0.x + s0.y) + (s1.x + s1.y);
+            }
+            tmem_wait_st();
+            // this warp's P is in TMEM; one arrival per warp on rank 0's barrier, and one
+            // on this CTA's
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_cluster(p_full0 + b * 8);
+                mbar_arrive(smem_u32(&bar->p_local[b]));
+            }
+        }
+        // ----------------------------------------------------------------- epilogue
+        // every P V is done (one commit after the last); the groups then add their sums
+        // under the final reference, the larger of theirs (references only rise)
+        if (ok && it.E > 0) ok = wait_all(smem_u32(&bar->o_final), 0);
+        if (ok) {
+            bar->fin_m[g][row] = m_seen;
+            bar->fin_l[g][row] = l;
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar->fin_bar));
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar->fin_bar), 0, abort_flag));
+        }
+        if (ok && blk < p.n_qblk) {
+            const float m0 = bar->fin_m[0][row], m1 = bar->fin_m[1][row];
+            const float m_fin = fmaxf(m0, m1);
+            const float lt = m_fin == -INFINITY
+                                 ? 0.f
+                                 : bar->fin_l[0][row] * fast_exp2(m0 - m_fin) +
+                                       bar->fin_l[1][row] * fast_exp2(m1 - m_fin);
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const size_t orow = ((size_t)it.h * p.nq_rows + (row_valid ? tok : 0)) * D + g * 64;
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {
+                uint32_t o[32];
+                if (it.E > 0) {
+                    tmem_ld32(tO + g * 64 + j * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
+                if (row_valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow +
+                                                           j * 32);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c]) * inv,
+                                                        __uint_as_float(o[8 * c + 1]) * inv),
+                                            pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv,
+                                                        __uint_as_float(o[8 * c + 3]) * inv),
+                                            pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv,
+                                                        __uint_as_float(o[8 * c + 5]) * inv),
+                                            pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv,
+                                                        __uint_as_float(o[8 * c + 7]) * inv));
+                }
+            }
+            if (row_valid && g == 0 && p.lse)
+                p.lse[(size_t)it.h * p.nq_rows + tok] =
+                    lt > 0.f ? (m_fin + log2f(lt)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && bar->abort && p.status) atomicExch(p.status, (int32_t)SVGA_ERR_TIMEOUT);
+    cluster_sync_all();  // no MMA of the pair and no remote arrival is still in flight
+    if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
 bool make_tmap(CUtensorMap *m, const void *base, int heads, int rows, int d, int box_rows)
 {
     EncodeTiledFn enc = get_encode_fn();
@@ -991,6 +1532,46 @@ svga_status launch_t(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("attention launch failed: %s", cudaGetErrorString(e));
+        return SVGA_ERR_CUDA;
+    }
+    return SVGA_OK;
+}
+
+// The pair kernel: plan mode, head_dim 128, 128-key chunks, bf16 output, K and V in
+// each head's order.  Two CTAs (one cluster) per work item.
+svga_status launch_pair(const AttnLaunch &a, const KParams &kp, cudaStream_t st)
+{
+    constexpr int D = pair::kD;
+    auto kfn = attn_fwd_pair_kernel;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kfn) != cudaSuccess) {
+        set_error("cudaFuncGetAttributes failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return SVGA_ERR_CUDA;
+    }
+    if (fa.numRegs < kRegsLaunch) {
+        set_error("pair attention kernel built with %d registers/thread, the register split "
+                  "needs %d",
+                  fa.numRegs, kRegsLaunch);
+        return SVGA_ERR_UNSUPPORTED;
+    }
+    CUtensorMap tq, tk64, tv;
+    if (!make_tmap(&tq, a.q, a.heads, a.nq_rows, D, kBlockM) ||
+        !make_tmap(&tk64, a.k, a.heads, a.nk_rows, D, 64) ||
+        !make_tmap(&tv, a.v, a.heads, a.nk_rows, D, pair::kKN)) {
+        set_error("cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+        return SVGA_ERR_CUDA;
+    }
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pair::kSmemLaunch) != cudaSuccess) {
+        set_error("cudaFuncSetAttribute(max dynamic shared memory) failed");
+        return SVGA_ERR_CUDA;
+    }
+    const int groups = (a.n_items + kp.num_parts - 1) / kp.num_parts;
+    if (groups > 0)
+        kfn<<<2 * groups, pair::kThreads, pair::kSmemLaunch, st>>>(tq, tk64, tv, kp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error("pair attention launch failed: %s", cudaGetErrorString(e));
         return SVGA_ERR_CUDA;
     }
     return SVGA_OK;
@@ -1114,6 +1695,13 @@ svga_status launch_attention(const AttnLaunch &a, void *stream)
     kp.part_o = split ? a.part_o : nullptr;
     kp.part_ml = split ? reinterpret_cast<float2 *>(a.part_ml) : nullptr;
     const int d = a.d, kn = a.kn;
+    if (a.cta_pair && a.mode == 0 && d == 128 && kn == 128 && !a.out_f32 && !a.kv_fm && !split) {
+        svga_status rc = launch_pair(a, kp, st);
+        if (rc != SVGA_OK) return rc;
+        KParams rest = kp;  // the items the pair kernel left
+        rest.pair_rest = 1;
+        return launch_t<128, 128, false>(a, rest, st);
+    }
     if (d == 128 && kn == 128)
         return a.out_f32 ? launch_t<128, 128, true>(a, kp, st) : launch_t<128, 128, false>(a, kp, st);
     if (d == 128 && kn == 64)

@@ -100,6 +100,7 @@ struct AttnLaunch {
     int test_stall;            // SVGA_FLAG_TEST_STALL: withhold the first K load
     int qo_fm;                 // SVGA_FLAG_QO_FRAME_MAJOR: q, o, lse frame-major
     int kv_fm;                 // SVGA_FLAG_KV_FRAME_MAJOR: k, v frame-major
+    int cta_pair;              // SVGA_FLAG_CTA_PAIR: work items on CTA pairs where it applies
     int kn;                    // keys per chunk: 64 or 128
     int tile_q, tile_k;        // plan mode: the problem's map tiles
     int check_plan;            // plan mode: compare the plan's header and items with the call

@@ -26,6 +26,7 @@ FLAG_NAIVE_B1 = 1
 FLAG_TILE_ALIGNED = 2
 FLAG_QO_FRAME_MAJOR = 4
 FLAG_KV_FRAME_MAJOR = 8
+FLAG_CTA_PAIR = 16
 FLAG_TEST_STALL = 1 << 16
 
 EXPORTED = ["svga_problem_rows", "svga_block_map_size", "svga_build_block_map",

@@ -99,6 +99,14 @@ enum {
      * permutation of K and V is not needed either.  With SVGA_FLAG_QO_FRAME_MAJOR no
      * tensor moves at all.  Results are identical bit for bit to the permuted call. */
     SVGA_FLAG_KV_FRAME_MAJOR = 8,
+    /* Run the work items on CTA pairs (two SMs, one tcgen05.mma over both blocks of an
+     * item, each SM holding half of every K and V chunk and two S tiles) instead of
+     * one CTA per item.  Same result within the tolerance, not bit for bit: the
+     * softmax takes its reference maximum per tile pair of visits differently.  Slower
+     * than the default on B200 at d = 128 (about 7 % at 75,600 tokens); kept for
+     * study.  Applies to head_dim 128 with 128-key chunks, bf16 K / V in each head's
+     * order (not with SVGA_FLAG_KV_FRAME_MAJOR); elsewhere the flag is ignored. */
+    SVGA_FLAG_CTA_PAIR = 16,
     /* Test hook for the failure path: the first K chunk of every CTA is never loaded,
      * so the kernel's bounded waits run out (about one second per CTA wave), every role
      * stops, copies in flight are drained, TMEM is released and map->status reads
@@ -279,7 +287,8 @@ SVGA_API svga_status svga_unpermute_tokens(const void *src, void *dst, const svg
  *                SVGA_ERR_INVALID_ARG and nothing is written (O and lse untouched)
  *   scale      : softmax scale, usually 1/sqrt(head_dim)
  *   flags      : 0 or a combination of SVGA_FLAG_NAIVE_B1 / SVGA_FLAG_TILE_ALIGNED
- *                (not both), SVGA_FLAG_QO_FRAME_MAJOR, SVGA_FLAG_KV_FRAME_MAJOR and the
+ *                (not both), SVGA_FLAG_QO_FRAME_MAJOR, SVGA_FLAG_KV_FRAME_MAJOR,
+ *                SVGA_FLAG_CTA_PAIR and the
  *                test hook
  *                SVGA_FLAG_TEST_STALL; other bits give SVGA_ERR_INVALID_ARG
  * bf16 inputs, fp32 accumulation and softmax, P rounded to bf16 for the PV product. */

@@ -163,6 +163,48 @@ def test_special_values():
         assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"Q=0 head {h}")
 
 
+@pytest.mark.parametrize("direction", [1, -1])
+def test_scores_rising_along_the_keys(direction):
+    """Q and K share one direction whose weight in K grows with the token index (down
+    to about -150, up to about +150 in units of the scaled score): with direction 1
+    each new tile lies far above the reference maximum the kernels take from the
+    first tile of a row, so the rescaling of O and of the running sums runs many times
+    per row (with -1 it never does).  Both kernels (one CTA, and a CTA pair) still
+    equal the oracle."""
+    wl = C.mid()
+    q, k, v, _, _, _ = inputs(wl)
+    q2, k2 = q.clone(), k.clone()
+    q2[..., 0] = 16.0
+    ramp = torch.linspace(-106.0, 106.0, wl.tokens) * direction
+    k2[..., 0] = ramp.to(torch.bfloat16)
+    o, lse, _ = run_sparse_path(wl, q2.cuda(), k2.cuda(), v.cuda())
+    rows = sample_rows(wl, 120, seed=11)
+    o = o.float().cpu().numpy()
+    lse = lse_to_frame_major(lse.cpu().numpy(), wl, wl.order)
+    for h in range(wl.heads):
+        ro, rl = oracle_rows(wl, q2, k2, v, h, rows)
+        assert_attn_close(o[h, rows], ro, lse[h, rows], rl, what=f"rising scores head {h}")
+    # the same through the one-CTA kernel (keys gathered from frame-major memory)
+    prob = svga.ProblemSpec.from_workload(wl)
+    bmap = svga.build_block_map(prob)
+    qd = q2.cuda()
+    qp = torch.empty_like(qd)
+    svga.svga_permute_tokens(qd, qp, prob)
+    op = torch.empty_like(qd)
+    lsep = torch.empty(wl.heads, wl.tokens, dtype=torch.float32, device="cuda")
+    svga.svga_sparse_attention_fwd(qp, k2.cuda(), v.cuda(), op, lsep, prob, bmap,
+                                   1.0 / math.sqrt(wl.head_dim), svga.FLAG_KV_FRAME_MAJOR)
+    o1 = torch.empty_like(qd)
+    svga.svga_unpermute_tokens(op, o1, prob)
+    torch.cuda.synchronize()
+    assert bmap.device_status() == 0
+    o1 = o1.float().cpu().numpy()
+    l1 = lse_to_frame_major(lsep.cpu().numpy(), wl, wl.order)
+    for h in range(wl.heads):
+        ro, rl = oracle_rows(wl, q2, k2, v, h, rows)
+        assert_attn_close(o1[h, rows], ro, l1[h, rows], rl, what=f"rising scores, one CTA, head {h}")
+
+
 def test_repeatable_bitwise():
     wl = C.mid()
     q, k, v, qd, kd, vd = inputs(wl)
