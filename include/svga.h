@@ -103,7 +103,7 @@ enum {
      * item, each SM holding half of every K and V chunk and two S tiles) instead of
      * one CTA per item.  Same result within the tolerance, not bit for bit: the
      * softmax takes its reference maximum per tile pair of visits differently.  Slower
-     * than the default on B200 at d = 128 (about 7 % at 75,600 tokens); kept for
+     * than the default on B200 at d = 128 (about 10 % at 75,600 tokens); kept for
      * study.  Applies to head_dim 128 with 128-key chunks, bf16 K / V in each head's
      * order (not with SVGA_FLAG_KV_FRAME_MAJOR); elsewhere the flag is ignored. */
     SVGA_FLAG_CTA_PAIR = 16,
