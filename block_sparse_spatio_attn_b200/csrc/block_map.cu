@@ -159,12 +159,20 @@ __device__ __forceinline__ int block_sum(int v, int *red)
     return t;
 }
 
-// One block per (q-tile, head): class of every k-tile and the row's two counts.
-__global__ void __launch_bounds__(256) classify_tiles_kernel(Geometry g, int anchor,
-                                                             const int4 *head_info, uint8_t *cls,
-                                                             int *full_cnt, int *bnd_cnt)
+// One block per (q-tile, head): class of every k-tile and the row's two counts.  The row
+// goes in segments of 256 groups of 8 k-tiles.  First each thread asks of one group
+// whether its key positions hold any pair the q-tile keeps: the rectangles of a range
+// cover exactly its tokens and the test is exact, so a group with none has 8 empty
+// tiles.  Then the threads classify the segment's tiles one by one, with the full test
+// only inside groups that hold a kept pair (about a third of them).
+constexpr int kGroupTiles = 8;
+constexpr int kClassifyThreads = 256;
+
+__global__ void __launch_bounds__(kClassifyThreads) classify_tiles_kernel(
+    Geometry g, int anchor, const int4 *head_info, uint8_t *cls, int *full_cnt, int *bnd_cnt)
 {
     __shared__ int red[8];
+    __shared__ uint8_t group_any[kClassifyThreads];
     const int i = blockIdx.x, h = blockIdx.y;
     const int4 hi = head_info[h];
     const int type = hi.x, band = hi.y, order = hi.z;
@@ -174,14 +182,14 @@ __global__ void __launch_bounds__(256) classify_tiles_kernel(Geometry g, int anc
     bool qpad = qa + g.tile_q > g.NP;
     Rect qr[4];
     const uint32_t qm = tile_rects(order, qa, qb, g.F, g.S, g.Sp, g.N, qr, qpad);
-    int nf = 0, nb = 0;
-    uint8_t *row = cls + ((size_t)h * g.n_q + i) * g.n_k;
-    for (int j = threadIdx.x; j < g.n_k; j += blockDim.x) {
-        const int ka = j * g.tile_k, kb = min(g.NP, ka + g.tile_k);
-        bool kpad = ka + g.tile_k > g.NP;
+    // does the q-tile keep any pair with the keys at positions [ka, kb)?  (all: all of
+    // them, holes aside)
+    auto test = [&](int ka, int kb, bool &all) {
+        bool kpad = false;
         Rect kr[4];
         const uint32_t km = tile_rects(order, ka, kb, g.F, g.S, g.Sp, g.N, kr, kpad);
-        bool full = !qpad && !kpad, any = false;
+        bool any = false;
+        all = !kpad;
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -189,13 +197,39 @@ __global__ void __launch_bounds__(256) classify_tiles_kernel(Geometry g, int anc
                 if (((qm >> a) & 1u) && ((km >> b) & 1u)) {
                     bool all_, any_;
                     rect_pair(type, band, anchor, qr[a], kr[b], all_, any_);
-                    full = full && all_;
+                    all = all && all_;
                     any = any || any_;
                 }
-        const uint8_t c = any ? (full ? 1 : 2) : 0;
-        row[j] = c;
-        nf += c == 1;
-        nb += c == 2;
+        return any;
+    };
+    int nf = 0, nb = 0;
+    uint8_t *row = cls + ((size_t)h * g.n_q + i) * g.n_k;
+    constexpr int kSegTiles = kClassifyThreads * kGroupTiles;
+    for (int seg = 0; seg < g.n_k; seg += kSegTiles) {
+        {
+            const int j0 = seg + threadIdx.x * kGroupTiles;
+            bool all_unused;
+            group_any[threadIdx.x] =
+                j0 < g.n_k &&
+                test(j0 * g.tile_k, min(g.NP, min(g.n_k, j0 + kGroupTiles) * g.tile_k), all_unused);
+        }
+        __syncthreads();
+        const int seg_end = min(g.n_k, seg + kSegTiles);
+        for (int j = seg + threadIdx.x; j < seg_end; j += kClassifyThreads) {
+            uint8_t c = 0;
+            if (group_any[(j - seg) / kGroupTiles]) {
+                const int ka = j * g.tile_k, kb = min(g.NP, ka + g.tile_k);
+                bool all;
+                const bool any = test(ka, kb, all);
+                // a tile reaching past the positions is never full
+                const bool full = all && !qpad && ka + g.tile_k <= g.NP;
+                c = any ? (full ? 1 : 2) : 0;
+            }
+            row[j] = c;
+            nf += c == 1;
+            nb += c == 2;
+        }
+        __syncthreads();  // group_any is rewritten by the next segment
     }
     nf = block_sum(nf, red);
     nb = block_sum(nb, red);
@@ -233,15 +267,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *cnt, int n, int *
     }
 }
 
-// Ordered stream compaction of one block's flags; returns this thread's slot and
-// the block total through *total.
-__device__ __forceinline__ int block_rank(bool flag, int *wsum, int *total)
+// Exclusive prefix sum over the block of one value per thread (warp shuffles, then the
+// warp totals); *total gets the block's sum.  Values may pack two 16-bit counts as long
+// as neither half overflows.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *wsum, int *total)
 {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const unsigned m = __ballot_sync(0xffffffffu, flag);
-    const int before = __popc(m & ((1u << lane) - 1u));
-    __syncthreads();
-    if (lane == 0) wsum[w] = __popc(m);
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+    }
+    __syncthreads();  // wsum may still be read by the previous call
+    if (lane == 31) wsum[w] = inc;
     __syncthreads();
     int off = 0, tot = 0;
     for (int i = 0; i < nw; ++i) {
@@ -249,8 +288,11 @@ __device__ __forceinline__ int block_rank(bool flag, int *wsum, int *total)
         tot += wsum[i];
     }
     *total = tot;
-    return off + before;
+    return off + inc - v;
 }
+
+// Elements a thread of the list and plan builders takes per step (consecutive ones).
+constexpr int kPerThread = 8;
 
 __global__ void __launch_bounds__(256) compact_lists_kernel(Geometry g, const uint8_t *cls,
                                                             const int *full_ptr, const int *bnd_ptr,
@@ -261,16 +303,32 @@ __global__ void __launch_bounds__(256) compact_lists_kernel(Geometry g, const ui
     const int i = blockIdx.x, h = blockIdx.y, r = h * g.n_q + i;
     const uint8_t *row = cls + (size_t)r * g.n_k;
     long long fo = full_ptr[r], bo = bnd_ptr[r];
-    for (int base = 0; base < g.n_k; base += blockDim.x) {
-        const int j = base + threadIdx.x;
-        const uint8_t c = j < g.n_k ? row[j] : 0;
-        int tf, tb;
-        const int pf = block_rank(c == 1, wsum, &tf);
-        if (c == 1 && fo + pf < full_cap) full_idx[fo + pf] = j;
-        const int pb = block_rank(c == 2, wsum, &tb);
-        if (c == 2 && bo + pb < bnd_cap) bnd_idx[bo + pb] = j;
-        fo += tf;
-        bo += tb;
+    // each step: kPerThread consecutive tiles per thread, one scan of both counts
+    for (int base = 0; base < g.n_k; base += blockDim.x * kPerThread) {
+        const int j0 = base + threadIdx.x * kPerThread;
+        uint8_t c[kPerThread];
+        int nf = 0, nb = 0;
+#pragma unroll
+        for (int u = 0; u < kPerThread; ++u) {
+            c[u] = j0 + u < g.n_k ? row[j0 + u] : 0;
+            nf += c[u] == 1;
+            nb += c[u] == 2;
+        }
+        int tot;
+        const int pos = block_exclusive_scan(nf | (nb << 16), wsum, &tot);
+        long long pf = fo + (pos & 0xFFFF), pb = bo + (pos >> 16);
+#pragma unroll
+        for (int u = 0; u < kPerThread; ++u) {
+            if (c[u] == 1) {
+                if (pf < full_cap) full_idx[pf] = j0 + u;
+                ++pf;
+            } else if (c[u] == 2) {
+                if (pb < bnd_cap) bnd_idx[pb] = j0 + u;
+                ++pb;
+            }
+        }
+        fo += tot & 0xFFFF;
+        bo += tot >> 16;
     }
 }
 
@@ -323,37 +381,46 @@ __global__ void __launch_bounds__(256) plan_write_kernel(Geometry g, const uint8
     const int item = blockIdx.x, h = item / g.n_pairs, p = item - h * g.n_pairs;
     const uint8_t *cls_h = cls + (size_t)h * g.n_q * g.n_k;
     long long off = item_off[item];
-    for (int base = 0; base < g.n_kc; base += blockDim.x) {
-        const int c = base + threadIdx.x;
-        const uint32_t e = c < g.n_kc ? entry_of(g, cls_h, p, c) : 0;
+    // each step: kPerThread consecutive chunks per thread, one scan of the entry counts
+    for (int base = 0; base < g.n_kc; base += blockDim.x * kPerThread) {
+        const int c0 = base + threadIdx.x * kPerThread;
+        uint32_t e[kPerThread];
+        int n = 0;
+#pragma unroll
+        for (int u = 0; u < kPerThread; ++u) {
+            e[u] = c0 + u < g.n_kc ? entry_of(g, cls_h, p, c0 + u) : 0u;
+            n += e[u] != 0;
+        }
         int tot;
-        const int pos = block_rank(e != 0, wsum, &tot);
-        if (e != 0 && off + pos < cap) entries[off + pos] = e;
+        long long pos = off + block_exclusive_scan(n, wsum, &tot);
+#pragma unroll
+        for (int u = 0; u < kPerThread; ++u)
+            if (e[u] != 0) {
+                if (pos < cap) entries[pos] = e[u];
+                ++pos;
+            }
         off += tot;
     }
 }
 
 // Longest-first order of the work items (ties: lower item index first), so that a
-// launch in plan order hands the long items out first.
+// launch in plan order hands the long items out first.  One warp per item counts the
+// items that go before it (a rank); the counts are read from L1.
 __global__ void __launch_bounds__(256) plan_sort_kernel(Geometry g, const int *item_cnt,
                                                         const int *item_off, int4 *items)
 {
-    __shared__ int tile[1024];
-    const int me = blockIdx.x * blockDim.x + threadIdx.x;
-    const int my = me < g.n_items ? item_cnt[me] : 0;
+    const int me = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (me >= g.n_items) return;  // whole warps leave together
+    const int my = item_cnt[me];
     int rank = 0;
-    for (int base = 0; base < g.n_items; base += 1024) {
-        __syncthreads();
-        for (int x = threadIdx.x; x < 1024; x += blockDim.x)
-            tile[x] = base + x < g.n_items ? item_cnt[base + x] : -1;
-        __syncthreads();
-        const int lim = min(1024, g.n_items - base);
-        for (int x = 0; x < lim; ++x) {
-            const int o = tile[x];
-            rank += (o > my) || (o == my && base + x < me);
-        }
+#pragma unroll 4
+    for (int o = lane; o < g.n_items; o += 32) {
+        const int x = __ldg(item_cnt + o);
+        rank += (x > my) || (x == my && o < me);
     }
-    if (me < g.n_items) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (lane == 0) {
         const int h = me / g.n_pairs, p = me - h * g.n_pairs;
         items[rank] = make_int4(h, 2 * p, item_off[me], my);
     }
@@ -423,7 +490,7 @@ svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svg
                               ((uint32_t)p->band[h] << 8);
         write_plan_header_kernel<<<(g.heads + 255) / 256, 256, 0, st>>>(hdr, local, head_info);
     }
-    classify_tiles_kernel<<<dim3(g.n_q, g.heads), 256, 0, st>>>(g, p->anchor_frame0, head_info,
+    classify_tiles_kernel<<<dim3(g.n_q, g.heads), kClassifyThreads, 0, st>>>(g, p->anchor_frame0, head_info,
                                                                 map->cls, full_cnt, bnd_cnt);
     scan_kernel<<<1, 1024, 0, st>>>(full_cnt, (int)rows, map->full_ptr, map->full_cap, map->status);
     scan_kernel<<<1, 1024, 0, st>>>(bnd_cnt, (int)rows, map->bnd_ptr, map->bnd_cap, map->status);
@@ -433,8 +500,8 @@ svga_status launch_build_block_map(const svga_problem *p, const Geometry &g, svg
     plan_count_kernel<<<g.n_items, 256, 0, st>>>(g, map->cls, item_cnt);
     scan_kernel<<<1, 1024, 0, st>>>(item_cnt, g.n_items, item_off, entry_cap, map->status);
     plan_write_kernel<<<g.n_items, 256, 0, st>>>(g, map->cls, item_off, entries, entry_cap);
-    // 64-thread blocks: the rank count is O(n) per item, so spread items over many SMs
-    plan_sort_kernel<<<(g.n_items + 63) / 64, 64, 0, st>>>(g, item_cnt, item_off, items);
+    // one warp per item
+    plan_sort_kernel<<<(g.n_items + 7) / 8, 256, 0, st>>>(g, item_cnt, item_off, items);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         set_error("block map launch failed: %s", cudaGetErrorString(e));
