@@ -161,10 +161,12 @@ __device__ __forceinline__ int block_sum(int v, int *red)
 
 // One block per (q-tile, head): class of every k-tile and the row's two counts.  The row
 // goes in segments of 256 groups of 8 k-tiles.  First each thread asks of one group
-// whether its key positions hold any pair the q-tile keeps: the rectangles of a range
-// cover exactly its tokens and the test is exact, so a group with none has 8 empty
-// tiles.  Then the threads classify the segment's tiles one by one, with the full test
-// only inside groups that hold a kept pair (about a third of them).
+// whether the q-tile keeps none, all or some of the pairs with its key positions: the
+// rectangles of a range cover exactly its tokens and the test is exact, so a group
+// with none has 8 empty tiles, and a group with all of them (and no position without
+// a token) has 8 full tiles, bar one reaching past the last position.  Then the threads
+// classify the segment's tiles, testing one by one only inside the mixed groups (those
+// at the edges of a band).
 constexpr int kGroupTiles = 8;
 constexpr int kClassifyThreads = 256;
 
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_tiles_kernel(
     Geometry g, int anchor, const int4 *head_info, uint8_t *cls, int *full_cnt, int *bnd_cnt)
 {
     __shared__ int red[8];
-    __shared__ uint8_t group_any[kClassifyThreads];
+    __shared__ uint8_t group_cls[kClassifyThreads];  // 0 none, 1 all, 2 some kept
     const int i = blockIdx.x, h = blockIdx.y;
     const int4 hi = head_info[h];
     const int type = hi.x, band = hi.y, order = hi.z;
@@ -208,17 +210,25 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_tiles_kernel(
     for (int seg = 0; seg < g.n_k; seg += kSegTiles) {
         {
             const int j0 = seg + threadIdx.x * kGroupTiles;
-            bool all_unused;
-            group_any[threadIdx.x] =
-                j0 < g.n_k &&
-                test(j0 * g.tile_k, min(g.NP, min(g.n_k, j0 + kGroupTiles) * g.tile_k), all_unused);
+            uint8_t gc = 0;
+            if (j0 < g.n_k) {
+                bool all;
+                if (test(j0 * g.tile_k, min(g.NP, min(g.n_k, j0 + kGroupTiles) * g.tile_k), all))
+                    gc = (all && !qpad) ? 1 : 2;
+            }
+            group_cls[threadIdx.x] = gc;
         }
         __syncthreads();
         const int seg_end = min(g.n_k, seg + kSegTiles);
         for (int j = seg + threadIdx.x; j < seg_end; j += kClassifyThreads) {
-            uint8_t c = 0;
-            if (group_any[(j - seg) / kGroupTiles]) {
-                const int ka = j * g.tile_k, kb = min(g.NP, ka + g.tile_k);
+            const uint8_t gc = group_cls[(j - seg) / kGroupTiles];
+            const int ka = j * g.tile_k;
+            uint8_t c = gc;
+            if (gc == 1) {
+                // every pair kept: full, unless the tile reaches past the positions
+                if (ka + g.tile_k > g.NP) c = 2;
+            } else if (gc == 2) {
+                const int kb = min(g.NP, ka + g.tile_k);
                 bool all;
                 const bool any = test(ka, kb, all);
                 // a tile reaching past the positions is never full
@@ -229,7 +239,7 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_tiles_kernel(
             nf += c == 1;
             nb += c == 2;
         }
-        __syncthreads();  // group_any is rewritten by the next segment
+        __syncthreads();  // group_cls is rewritten by the next segment
     }
     nf = block_sum(nf, red);
     nb = block_sum(nb, red);
