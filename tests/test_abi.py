@@ -190,7 +190,9 @@ def test_sparse_forward_flag_and_part_checks_on_the_host(lib):
     fm = svga.FLAG_QO_FRAME_MAJOR | svga.FLAG_KV_FRAME_MAJOR
     for flags in (0, svga.FLAG_NAIVE_B1, svga.FLAG_TILE_ALIGNED, svga.FLAG_QO_FRAME_MAJOR,
                   svga.FLAG_KV_FRAME_MAJOR, fm, fm | svga.FLAG_NAIVE_B1,
-                  fm | svga.FLAG_TILE_ALIGNED, fm | svga.FLAG_TEST_STALL):
+                  fm | svga.FLAG_TILE_ALIGNED, fm | svga.FLAG_TEST_STALL, svga.FLAG_CTA_PAIR,
+                  svga.FLAG_CTA_PAIR | svga.FLAG_QO_FRAME_MAJOR | svga.FLAG_NAIVE_B1,
+                  svga.FLAG_CTA_PAIR | svga.FLAG_TEST_STALL):
         assert call(flags, scale=-1.0) == 1, flags
         assert b"scale" in lib.svga_last_error(), flags
     assert call(0, part=2, n=2) == 1 and b"part" in lib.svga_last_error()
