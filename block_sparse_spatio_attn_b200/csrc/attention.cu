@@ -189,7 +189,7 @@ __device__ __forceinline__ int plan_item_of_block(const KParams &p)
 // A caller's plan must describe this launch before any of its offsets is used: the
 // header against the launch's shape, tiles, anchor and item count, then this CTA's work
 // item (head, even first block, entry range inside the plan) and the head's info.
-// Every thread of the CTA reads the same words, so the verdict is uniform.
+// Every thread of the CTA reads the same words, so the outcome is uniform.
 __device__ __forceinline__ bool plan_matches(const KParams &p, int kn, int slot)
 {
     const int4 *h4 = reinterpret_cast<const int4 *>(p.hdr);
