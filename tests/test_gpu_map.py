@@ -14,6 +14,7 @@ if not torch.cuda.is_available():
 
 from block_sparse_spatio_attn_b200 import svga  # noqa: E402
 from tests.helpers import problem_of  # noqa: E402
+from tests.test_oracle_tile_counts import HEADLINE, TWOK  # noqa: E402
 
 
 def oracle_flat_map(wl, order, tq, tk, heads=None):
@@ -192,3 +193,26 @@ def test_validator_rejects_corrupted_maps(what, msg):
     with pytest.raises(svga.SvgaError) as e:
         svga.svga_validate_block_map(prob, bmap)
     assert e.value.status == 1 and msg in str(e.value), str(e.value)
+
+
+def _pinned(rows, name):
+    """(full, boundary, empty) of the named row of an independent tile-count table."""
+    return tuple(next(c[7:10] for c in rows if c[0] == name))
+
+
+@pytest.mark.parametrize("name", ["headline", "2k"])
+def test_map_counts_equal_the_independent_integers(name):
+    """The GPU map of the whole workload (tile 128x128) has, head by head, the (full,
+    boundary, empty) tile counts that were computed independently of this library and
+    that the oracle reproduces (tests/test_oracle_tile_counts.py): spatial heads
+    frame-major, temporal heads in the anchor-first temporal-major order."""
+    if name == "headline":
+        rows, sp, tp = HEADLINE, "headline spatial FM 128", "headline temporal anchor-first 128"
+    else:
+        rows, sp, tp = TWOK, "2k spatial FM 128", "2k temporal anchor-first 128"
+    expect = {C.SPATIAL: _pinned(rows, sp), C.TEMPORAL: _pinned(rows, tp)}
+    wl = C.ALL[name]()
+    _, cls, *_ = gpu_map(wl, None, 128, 128)
+    for h in range(wl.heads):
+        got = tuple(int((cls[h] == c).sum()) for c in (1, 2, 0))
+        assert got == expect[wl.head_type[h]], (name, h, got)
